@@ -1,0 +1,254 @@
+// extern "C" entry points of libfp4 (declared in include/fp4.h): host-side
+// argument checks, then kernel launches on the caller's stream.
+
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "fp4_internal.h"
+
+namespace fp4 {
+
+cudaError_t device_info(DeviceInfo* out)
+{
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev].sm_count > 0) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    DeviceInfo d;
+    e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) cache[dev] = d;
+    *out = d;
+    return cudaSuccess;
+}
+
+thread_local char g_last_error[256] = "";
+
+void set_last_error(const char* what, cudaError_t e)
+{
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s", what,
+             e == cudaSuccess ? "invalid argument" : cudaGetErrorString(e));
+}
+
+}  // namespace fp4
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_fmt(fp4_format f) { return f == FP4_NVFP4 || f == FP4_MXFP4; }
+
+fp4_status from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return FP4_OK;
+    if (e == cudaErrorNoDevice || e == cudaErrorInsufficientDriver) return FP4_ERR_NO_DEVICE;
+    return FP4_ERR_CUDA;
+}
+
+// The kernels use tcgen05 / TMA instructions of sm_100a.
+fp4_status require_device(fp4::DeviceInfo* dev)
+{
+    cudaError_t e = fp4::device_info(dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return from_cuda(e);
+    }
+    if (dev->major != 10) return FP4_ERR_NO_DEVICE;
+    return FP4_OK;
+}
+
+constexpr int64_t kMaxGridY = 65535;
+constexpr int64_t kMaxRows = (int64_t)1 << 31;
+
+}  // namespace
+
+extern "C" {
+
+int fp4_abi_version(void) { return 1; }
+
+const char* fp4_last_error(void) { return fp4::g_last_error; }
+
+const char* fp4_status_string(fp4_status s)
+{
+    switch (s) {
+    case FP4_OK: return "FP4_OK";
+    case FP4_ERR_INVALID_ARG: return "FP4_ERR_INVALID_ARG";
+    case FP4_ERR_UNSUPPORTED_SHAPE: return "FP4_ERR_UNSUPPORTED_SHAPE";
+    case FP4_ERR_MISALIGNED: return "FP4_ERR_MISALIGNED";
+    case FP4_ERR_CUDA: return "FP4_ERR_CUDA";
+    case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT";
+    case FP4_ERR_NO_DEVICE: return "FP4_ERR_NO_DEVICE";
+    }
+    return "FP4_ERR_UNKNOWN";
+}
+
+size_t fp4_packed_bytes(int64_t rows, int64_t k)
+{
+    if (rows <= 0 || k <= 0) return 0;
+    return (size_t)rows * (size_t)(k / 2);
+}
+
+size_t fp4_scale_bytes(fp4_format fmt, int64_t rows, int64_t k)
+{
+    if (!valid_fmt(fmt) || rows <= 0 || k <= 0) return 0;
+    const int64_t nsc = k / fp4::block_size(fmt);
+    return (size_t)((rows + 127) / 128) * (size_t)((nsc + 3) / 4) * 512u;
+}
+
+fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                    float* gs_out, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (rows < 0 || cols < 0 || gs_out == nullptr) return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && in_bf16 == nullptr) return FP4_ERR_INVALID_ARG;
+    if (ld < cols) return FP4_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld % 8 != 0 || !aligned16(in_bf16) || (reinterpret_cast<uintptr_t>(gs_out) & 3u))
+        return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_amax(static_cast<const uint16_t*>(in_bf16), rows, cols, ld, gs_out,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int64_t rows,
+                        int64_t cols, int64_t ld, void* packed_out, void* scales_out,
+                        const float* global_scale, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_fmt(fmt) || (axis != FP4_ROWWISE && axis != FP4_COLWISE)) return FP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols) return FP4_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return FP4_OK;
+    if (!in_bf16 || !packed_out || !scales_out) return FP4_ERR_INVALID_ARG;
+    if (fmt == FP4_NVFP4 && !global_scale) return FP4_ERR_INVALID_ARG;
+    const int kb = fp4::block_size(fmt);
+    if (axis == FP4_ROWWISE) {
+        if (cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if ((rows + 127) / 128 > kMaxGridY) return FP4_ERR_UNSUPPORTED_SHAPE;
+    } else {
+        if (rows % (4 * kb) != 0 || cols % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if ((cols + 127) / 128 > kMaxGridY) return FP4_ERR_UNSUPPORTED_SHAPE;
+    }
+    if (ld % 8 != 0 || !aligned16(in_bf16) || !aligned16(packed_out) || !aligned16(scales_out))
+        return FP4_ERR_MISALIGNED;
+    if (global_scale && (reinterpret_cast<uintptr_t>(global_scale) & 3u)) return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_quantize(
+        (int)fmt, (int)axis, static_cast<const uint16_t*>(in_bf16), rows, cols, ld,
+        static_cast<uint8_t*>(packed_out), static_cast<uint8_t*>(scales_out),
+        fmt == FP4_NVFP4 ? global_scale : nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, float* alpha_out,
+                                        fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!gsA || !gsB || !alpha_out) return FP4_ERR_INVALID_ARG;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_alpha(gsA, gsB, alpha_out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K)
+{
+    if (!valid_fmt(fmt)) return 0;
+    fp4::DeviceInfo dev;
+    if (fp4::device_info(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
+}
+
+fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, const void* B,
+                                const void* sB, int64_t M, int64_t N, int64_t K,
+                                const float* alpha, void* D, int64_t ldd, void* workspace,
+                                size_t ws_bytes, fp4_gemm_kernel kernel, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_fmt(fmt)) return FP4_ERR_INVALID_ARG;
+    if (kernel != FP4_GEMM_AUTO && kernel != FP4_GEMM_PREFILL && kernel != FP4_GEMM_DECODE)
+        return FP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return FP4_OK;
+    if (!D) return FP4_ERR_INVALID_ARG;
+    const int kq = fmt == FP4_NVFP4 ? 64 : 128;
+    if (K % kq != 0 || N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= kMaxRows || N >= kMaxRows || K / 2 >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldd % 8 != 0 || !aligned16(D)) return FP4_ERR_MISALIGNED;
+    if (K > 0) {
+        if (!A || !sA || !B || !sB) return FP4_ERR_INVALID_ARG;
+        if (!aligned16(A) || !aligned16(B) || !aligned16(sA) || !aligned16(sB))
+            return FP4_ERR_MISALIGNED;
+    }
+    if (alpha && (reinterpret_cast<uintptr_t>(alpha) & 3u)) return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        return from_cuda(cudaMemset2DAsync(D, (size_t)ldd * 2, 0, (size_t)N * 2, (size_t)M, s));
+    }
+    if (!fp4::tensor_map_encoder_available()) return FP4_ERR_NO_DEVICE;
+
+    const size_t need = fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
+    bool decode = false;
+    if (kernel == FP4_GEMM_DECODE) {
+        if (M > 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (!workspace || ws_bytes < need) return FP4_ERR_INVALID_ARG;
+        if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+        decode = true;
+    } else if (kernel == FP4_GEMM_AUTO) {
+        decode = M <= 16 && workspace && ws_bytes >= need && aligned16(workspace);
+    }
+    fp4::GemmArgs a;
+    a.fmt = (int)fmt;
+    a.A = static_cast<const uint8_t*>(A);
+    a.sA = static_cast<const uint8_t*>(sA);
+    a.B = static_cast<const uint8_t*>(B);
+    a.sB = static_cast<const uint8_t*>(sB);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.alpha = alpha;
+    a.D = static_cast<uint16_t*>(D);
+    a.ldd = ldd;
+    a.ws = workspace;
+    a.ws_bytes = ws_bytes;
+    const cudaError_t e = decode ? fp4::launch_gemm_decode(a, dev, s) : fp4::launch_gemm_prefill(a, dev, s);
+    return from_cuda(e);
+}
+
+fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B, const void* sB,
+                    int64_t M, int64_t N, int64_t K, const float* alpha, void* D, int64_t ldd,
+                    void* workspace, size_t ws_bytes, fp4_stream_t stream)
+{
+    return fp4_gemm_with_kernel(fmt, A, sA, B, sB, M, N, K, alpha, D, ldd, workspace, ws_bytes,
+                                FP4_GEMM_AUTO, stream);
+}
+
+fp4_status fp4_get_device_status(fp4_stream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return from_cuda(e);
+    unsigned int word = 0;
+    e = fp4::read_and_clear_error_word(&word);
+    if (e != cudaSuccess) return from_cuda(e);
+    return word ? FP4_ERR_TIMEOUT : FP4_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Host-side declarations shared by the translation units of libfp4.
+#pragma once
+
+#include <cstdint>
+#include <cstddef>
+#include <cuda_runtime.h>
+
+#include "../../include/fp4.h"
+
+namespace fp4 {
+
+constexpr int kNv = 0;
+constexpr int kMx = 1;
+
+inline int block_size(int fmt) { return fmt == kMx ? 32 : 16; }
+
+// Device properties cached per device ordinal.
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0;
+    int minor = 0;
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// quantize.cu
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                        float* gs_out, cudaStream_t s);
+cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s);
+cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
+                            int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
+                            cudaStream_t s);
+
+// gemm.cu
+struct GemmArgs {
+    int fmt;
+    const uint8_t* A;   // [M x K/2]
+    const uint8_t* sA;
+    const uint8_t* B;   // [N x K/2]
+    const uint8_t* sB;
+    int64_t M, N, K;
+    const float* alpha;
+    uint16_t* D;        // bf16 [M x N], ldd
+    int64_t ldd;
+    void* ws;
+    size_t ws_bytes;
+};
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
+cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
+cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
+cudaError_t read_and_clear_error_word(unsigned int* word);
+int tensor_map_encoder_available();
+
+// Records the detail of a failure for fp4_last_error() (thread-local).
+void set_last_error(const char* what, cudaError_t e);
+extern thread_local char g_last_error[256];
+
+}  // namespace fp4

@@ -1,0 +1,792 @@
+// W4A4 block-scaled GEMM on the 5th-generation tensor cores (sm_100a):
+// D = alpha * A_hat * B_hat^T, A_hat/B_hat = E2M1 codes times per-block scales.
+//
+// Method: "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell",
+// "2. Hardware-Managed Tensor Core Dot-Products" (TMA streams the packed
+// 4-bit tiles and their scale vectors into shared memory; the tensor core
+// forms the block dot products, multiplies them by S_u * S_v and accumulates
+// in FP32) and "How Microscaling FP4 (MXFP4) Halves Memory Bandwidth...",
+// "Silicon Execution" (accumulate in 32-bit precision before storing).
+//
+// Kernel structure (one CTA per SM, persistent):
+//   warp 0      TMA producer: packed A/B tiles via tensor maps (128-byte
+//               swizzle), scale chunks via 1-D bulk copies, into a ring of
+//               STAGES shared-memory stages guarded by full/empty mbarriers.
+//   warp 1      TMEM allocation; one thread issues tcgen05.cp (scales,
+//               shared -> tensor memory) and tcgen05.mma (kind::mxf4nvf4,
+//               block_scale, 128 x BN x 64 per instruction), then
+//               tcgen05.commit to release stages and to publish the
+//               accumulator.
+//   warps 2-5   epilogue: tcgen05.ld of the FP32 accumulator (each warp its
+//               32-lane quadrant), alpha, BF16 round-to-nearest-even, 16-byte
+//               stores; or FP32 split-K partials (decode form).
+// Every mbarrier wait is bounded by %globaltimer; on expiry the CTA sets the
+// library's device error word, stops issuing work, drains what it already
+// issued, frees its tensor memory and returns (no trap).
+//
+// Scale layout in tensor memory: one 512-byte chunk (128 rows x 4 scale
+// bytes, the global tile layout) is copied with tcgen05.cp 32x128b.warpx4 to
+// 4 TMEM columns; column c, lane l then holds the 4 scale bytes of row
+// 32c + l (replicated over the four lane quadrants).  For NVFP4
+// (scale_vec::4X, E4M3) one chunk serves one K=64 MMA; for MXFP4
+// (scale_vec::2X, E8M0) one chunk serves two, selected by scale-factor id 0/2.
+//
+// Decode form (M <= 16 tokens): the operands are swapped so that the weight
+// rows fill the 128-row MMA side and the tokens form a 16-wide N side; the
+// (weight tile, K stage) work units are split evenly over the CTAs
+// (stream-K), each CTA writes FP32 partials per weight tile it touched, and a
+// reduction kernel sums them in a fixed order, applies alpha and writes BF16.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "fp4_internal.h"
+
+namespace fp4 {
+
+__device__ unsigned int g_fp4_error_word;
+
+namespace {
+
+constexpr int BM = 128;             // MMA M (rows of the A-side operand per tile)
+constexpr int BK = 256;             // K elements per pipeline stage (128 bytes/row)
+constexpr int BK_BYTES = BK / 2;
+constexpr int MMA_K = 64;           // K per tcgen05.mma for FP4
+constexpr int A_BYTES = BM * BK_BYTES;
+constexpr int SF_CHUNK = 512;       // 128 rows x 4 scale bytes
+constexpr int SFA_BYTES = 4 * SF_CHUNK;
+constexpr int kThreads = 192;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+enum : unsigned { ERR_FULL = 1u, ERR_EMPTY = 2u, ERR_ACC_FULL = 4u, ERR_ACC_EMPTY = 8u,
+                  ERR_DRAIN = 16u };
+
+template <int BN, int STAGES>
+struct Cfg {
+    static constexpr int BH = (BN + 127) / 128;          // 128-row scale tiles of B per tile
+    static constexpr int B_BYTES = BN * BK_BYTES;
+    static constexpr int SFB_BYTES = BH * SFA_BYTES;
+    static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+    static constexpr int OFF_B = A_BYTES;
+    static constexpr int OFF_SFA = A_BYTES + B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    static constexpr int SF_COL0 = BN < 32 ? 32 : BN;    // first TMEM column of the scale ring
+    static constexpr int SFA_COLS = 4 * 4;               // 4 chunks x 4 columns
+    static constexpr int SF_COLS = SFA_COLS + 4 * 4 * BH;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
+    static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+    static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
+};
+
+struct Params {
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    int32_t rows_a, rows_b, K;
+    int32_t ks_total;          // K stages per tile
+    int32_t sf_col_tiles;      // 512-byte scale tiles per 128-row group
+    int32_t sfa_row_tiles, sfb_row_tiles;
+    int32_t tiles_m, tiles_n;
+    int32_t units;             // stream-K: tiles_m * ks_total
+    int32_t max_seg;           // stream-K: partial slots per CTA
+    const float* alpha;
+    uint16_t* D;
+    int64_t ldd;
+    float* ws;
+};
+
+// ------------------------------------------------------------------------
+// PTX wrappers
+// ------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t now_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `bar` with the given parity.  Gives up when another
+// role has raised the CTA's abort flag or after kTimeoutNs; in the latter
+// case raises the flag and records `code` in the device error word.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned code)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = now_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort_flag) return false;
+            if (now_ns() - t0 > kTimeoutNs) {
+                *abort_flag = 1;
+                atomicOr(&g_fp4_error_word, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Wait that ignores the abort flag (used only to drain work already issued).
+__device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity)
+{
+    const uint64_t t0 = now_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (now_ns() - t0 > kTimeoutNs) {
+            atomicOr(&g_fp4_error_word, ERR_DRAIN);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint32_t bar, uint32_t dst,
+                                            int32_t x, int32_t y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+template <bool MX>
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    if (MX) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::2X"
+            " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+            " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    }
+}
+
+// Shared-memory matrix descriptor: K-major rows of 128 bytes with the
+// 128-byte swizzle, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Descriptor of one 512-byte scale chunk: 32 rows of 16 bytes, no swizzle,
+// 8-row groups 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with block scaling: E2M1 x E2M1,
+// FP32 accumulate, K-major A and B, M = 128, N = BN; scale type UE8M0 (MX) or
+// UE4M3 (NV); sf_id selects the scale byte pair (2X) inside each column.
+template <int BN, bool MX>
+__device__ __forceinline__ uint32_t make_idesc(uint32_t sf_id)
+{
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+           ((MX ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Completes outstanding tcgen05.ld; the registers are threaded through so
+// that no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ------------------------------------------------------------------------
+// Work schedule shared by the three roles.  A segment is a run of K stages
+// of one output tile.
+// ------------------------------------------------------------------------
+struct Seg {
+    int tm, tn, kb, ke, slot;
+};
+
+template <bool STREAM_K>
+struct Schedule {
+    const Params& p;
+    int next_tile;   // prefill: next tile index
+    int u, ue, ub;   // stream-K: unit cursor / range
+    __device__ explicit Schedule(const Params& pp) : p(pp)
+    {
+        if (STREAM_K) {
+            const int64_t G = gridDim.x;
+            ub = (int)(((int64_t)blockIdx.x * p.units) / G);
+            ue = (int)(((int64_t)(blockIdx.x + 1) * p.units) / G);
+            u = ub;
+        } else {
+            next_tile = blockIdx.x;
+        }
+    }
+    __device__ bool next(Seg& s)
+    {
+        if (STREAM_K) {
+            if (u >= ue) return false;
+            s.tm = u / p.ks_total;
+            s.tn = 0;
+            s.kb = u % p.ks_total;
+            const int left = ue - u;
+            s.ke = min(p.ks_total, s.kb + left);
+            s.slot = s.tm - ub / p.ks_total;
+            u += s.ke - s.kb;
+            return true;
+        } else {
+            if (next_tile >= p.tiles_m * p.tiles_n) return false;
+            s.tm = next_tile % p.tiles_m;
+            s.tn = next_tile / p.tiles_m;
+            s.kb = 0;
+            s.ke = p.ks_total;
+            s.slot = 0;
+            next_tile += gridDim.x;
+            return true;
+        }
+    }
+};
+
+// ------------------------------------------------------------------------
+// The kernel
+// ------------------------------------------------------------------------
+template <int BN, int STAGES, bool MX, bool STREAM_K>
+__global__ void __launch_bounds__(kThreads, 1)
+fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const Params p)
+{
+    using C = Cfg<BN, STAGES>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+    // bars[0..S): full, bars[S..2S): empty, bars[2S]: acc_full,
+    // bars[2S+1]: acc_empty, bars[2S+2]: drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t smem0 = smem_u32(smem);
+    auto full = [&](int s) { return smem_u32(&bars[s]); };
+    auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
+    const uint32_t acc_full = smem_u32(&bars[2 * STAGES]);
+    const uint32_t acc_empty = smem_u32(&bars[2 * STAGES + 1]);
+    const uint32_t drain = smem_u32(&bars[2 * STAGES + 2]);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full(s), 1);
+            mbar_init(empty(s), 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 4);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            Schedule<STREAM_K> sched(p);
+            Seg sg;
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            while (ok && sched.next(sg)) {
+                // scale row tiles of B that exist for this tile
+                int nbh = 0;
+                const int rtb0 = (sg.tn * BN) / 128;
+                for (int h = 0; h < C::BH; ++h)
+                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
+                for (int ks = sg.kb; ks < sg.ke; ++ks) {
+                    if (!wait_bounded(empty(stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const int k0 = ks * BK;
+                    const int nk = min(4, (p.K - k0) / MMA_K);
+                    const int nch = MX ? nk / 2 : nk;
+                    const int ct0 = MX ? k0 / 128 : k0 / 64;
+                    const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
+                    const uint32_t st = smem0 + stage * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(full(stage), A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
+                    tma_load_2d(&tmA, full(stage), st, k0 / 2, sg.tm * BM);
+                    tma_load_2d(&tmB, full(stage), st + C::OFF_B, k0 / 2, sg.tn * BN);
+                    bulk_load(st + C::OFF_SFA,
+                              p.sfa + ((int64_t)sg.tm * p.sf_col_tiles + ct0) * SF_CHUNK, sf_bytes,
+                              full(stage));
+                    for (int h = 0; h < nbh; ++h)
+                        bulk_load(st + C::OFF_SFB + h * SFA_BYTES,
+                                  p.sfb + ((int64_t)(rtb0 + h) * p.sf_col_tiles + ct0) * SF_CHUNK,
+                                  sf_bytes, full(stage));
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Drain: the last min(issued, STAGES) stages may still be in flight
+            // if the consumer stopped early; wait for their transactions.
+            if (!ok || *abort_flag) {
+                const int n = issued < STAGES ? issued : STAGES;
+                for (int i = 1; i <= n; ++i) {
+                    int s = stage - i;
+                    uint32_t ph = phase;
+                    if (s < 0) {
+                        s += STAGES;
+                        ph ^= 1u;
+                    }
+                    wait_drain(full(s), ph);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            Schedule<STREAM_K> sched(p);
+            Seg sg;
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            while (ok && sched.next(sg)) {
+                if (!wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
+                tc_fence_after();
+                const int rtb0 = (sg.tn * BN) / 128;
+                int nbh = 0;
+                for (int h = 0; h < C::BH; ++h)
+                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
+                for (int ks = sg.kb; ks < sg.ke; ++ks) {
+                    if (!wait_bounded(full(stage), phase, abort_flag, ERR_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int k0 = ks * BK;
+                    const int nk = min(4, (p.K - k0) / MMA_K);
+                    const int nch = MX ? nk / 2 : nk;
+                    const uint32_t st = smem0 + stage * C::STAGE_BYTES;
+                    const uint32_t tsf = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
+                    const uint32_t tsfb = tsf + C::SFA_COLS;
+                    for (int j = 0; j < nch; ++j) {
+                        tc_cp_sf(tsf + 4 * j, desc_sf(st + C::OFF_SFA + j * SF_CHUNK));
+                        for (int h = 0; h < nbh; ++h)
+                            tc_cp_sf(tsfb + (j * C::BH + h) * 4,
+                                     desc_sf(st + C::OFF_SFB + h * SFA_BYTES + j * SF_CHUNK));
+                    }
+                    for (int j = 0; j < nk; ++j) {
+                        const int chunk = MX ? (j >> 1) : j;
+                        const uint32_t sf_id = MX ? (uint32_t)((j & 1) * 2) : 0u;
+                        const uint64_t ad = desc_sw128(st + j * 32);
+                        const uint64_t bd = desc_sw128(st + C::OFF_B + j * 32);
+                        tc_mma<MX>(tmem_base, ad, bd, make_idesc<BN, MX>(sf_id), tsf + 4 * chunk,
+                                   tsfb + chunk * C::BH * 4, (ks > sg.kb || j > 0) ? 1u : 0u);
+                    }
+                    tc_commit(empty(stage));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(acc_full);
+                acc_phase ^= 1u;
+            }
+            // make sure every tcgen05 operation issued here has completed
+            tc_commit(drain);
+            wait_drain(drain, 0);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;               // TMEM lane quadrant of this warp
+        const int row = q * 32 + lane;        // accumulator row of this thread
+        const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+        Schedule<STREAM_K> sched(p);
+        Seg sg;
+        uint32_t acc_phase = 0;
+        while (sched.next(sg)) {
+            // lane 0 polls, the warp follows it as a whole so that the
+            // .sync.aligned tensor-memory loads below stay warp-uniform
+            int ok = 0;
+            if (lane == 0) ok = wait_bounded(acc_full, acc_phase, abort_flag, ERR_ACC_FULL) ? 1 : 0;
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            __syncwarp();
+            tc_fence_after();
+            if (!STREAM_K) {
+                const int64_t gm = (int64_t)sg.tm * BM + row;
+                const bool row_ok = gm < p.rows_a;
+                uint16_t* drow = p.D + gm * p.ldd;
+#pragma unroll 1
+                for (int c = 0; c < BN / 16; ++c) {
+                    uint32_t r[16];
+                    tmem_ld16(trow + c * 16, r);
+                    tmem_wait_ld(r);
+                    const int gn0 = sg.tn * BN + c * 16;
+                    if (row_ok) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int gn = gn0 + 8 * h;
+                            if (gn < p.rows_b) {
+                                uint4 o;
+                                o.x = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 0])),
+                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 1])));
+                                o.y = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 2])),
+                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 3])));
+                                o.z = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 4])),
+                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 5])));
+                                o.w = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 6])),
+                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 7])));
+                                *reinterpret_cast<uint4*>(drow + gn) = o;
+                            }
+                        }
+                    }
+                }
+            } else {
+                float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
+#pragma unroll 1
+                for (int c = 0; c < BN / 16; ++c) {
+                    uint32_t r[16];
+                    tmem_ld16(trow + c * 16, r);
+                    tmem_wait_ld(r);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        slot[(c * 16 + j) * BM + row] = __uint_as_float(r[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+            acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// Sum of the stream-K partials of each output element in CTA order, times
+// alpha, to BF16.  Output D[m][n] (m < tokens, n < weight rows).
+template <int BN>
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int max_seg, int units, int G,
+                                     int ks_total, int n_rows, int tokens,
+                                     const float* __restrict__ alpha_ptr, uint16_t* __restrict__ D,
+                                     int64_t ldd)
+{
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)n_rows * tokens) return;
+    const int n = (int)(idx % n_rows);
+    const int m = (int)(idx / n_rows);
+    const int tm = n / BM, lane = n % BM;
+    const int64_t x0 = (int64_t)tm * ks_total, x1 = x0 + ks_total - 1;
+    const int c0 = (int)(((x0 + 1) * G - 1) / units);
+    const int c1 = (int)(((x1 + 1) * G - 1) / units);
+    float sum = 0.0f;
+    for (int c = c0; c <= c1; ++c) {
+        const int ubc = (int)(((int64_t)c * units) / G);
+        const int slot = tm - ubc / ks_total;
+        sum = __fadd_rn(sum, ws[(((int64_t)c * max_seg + slot) * BN + m) * BM + lane]);
+    }
+    const float a = alpha_ptr ? __ldg(alpha_ptr) : 1.0f;
+    const float v = __fmul_rn(a, sum);
+    uint32_t b = pack_bf16x2(v, 0.0f);
+    D[(int64_t)m * ldd + n] = (uint16_t)(b & 0xFFFFu);
+}
+
+// ------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
+
+// 2-D map over a packed operand [rows x row_bytes] (uint8), box 128 bytes x
+// box_rows, 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows)
+{
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Raises the kernel's dynamic shared-memory limit once per device; the
+// statics are distinct for every instantiation of the kernel template.
+template <int BN, int STAGES, bool MX, bool STREAM_K>
+cudaError_t set_smem_once(int bytes)
+{
+    static std::mutex mu;
+    static uint64_t done_mask = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && ((done_mask >> dev) & 1ull)) return cudaSuccess;
+    e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev < 64) done_mask |= 1ull << dev;
+    return e;
+}
+
+template <int BN, int STAGES, bool MX, bool STREAM_K>
+cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid,
+                          cudaStream_t s)
+{
+    using C = Cfg<BN, STAGES>;
+    cudaError_t e = set_smem_once<BN, STAGES, MX, STREAM_K>(C::SMEM);
+    if (e != cudaSuccess) {
+        set_last_error("cudaFuncSetAttribute(max dynamic shared memory)", e);
+        return e;
+    }
+    fp4_gemm_kernel<BN, STAGES, MX, STREAM_K><<<grid, kThreads, C::SMEM, s>>>(ta, tb, p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        cudaFuncAttributes fa{};
+        cudaFuncGetAttributes(&fa, fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>);
+        int dev = 0, optin = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        cudaGetLastError();
+        char buf[200];
+        snprintf(buf, sizeof buf,
+                 "GEMM kernel launch (grid %d, smem %d, optin %d, func max dyn %d, static %zu, regs %d)",
+                 grid, C::SMEM, optin, fa.maxDynamicSharedSizeBytes, fa.sharedSizeBytes, fa.numRegs);
+        set_last_error(buf, e);
+    }
+    return e;
+}
+
+constexpr int PREFILL_BN = 256, PREFILL_STAGES = 4;
+constexpr int DECODE_BN = 16, DECODE_STAGES = 8;
+
+int decode_max_seg(int units, int G, int ks_total)
+{
+    const int span = (units + G - 1) / G;
+    return (span - 1) / ks_total + 2;
+}
+
+}  // namespace
+
+int tensor_map_encoder_available() { return encoder() != nullptr; }
+
+size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count)
+{
+    if (M > DECODE_BN || M <= 0 || N <= 0 || K <= 0 || sm_count <= 0) return 0;
+    const int ks_total = (int)((K + BK - 1) / BK);
+    const int units = (int)((N + BM - 1) / BM) * ks_total;
+    const int G = sm_count < units ? sm_count : units;
+    return (size_t)G * decode_max_seg(units, G, ks_total) * DECODE_BN * BM * sizeof(float);
+}
+
+static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t rows_b,
+                        const uint8_t* sfa, const uint8_t* sfb)
+{
+    const int kb = block_size(a.fmt);
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.rows_a = (int32_t)rows_a;
+    p.rows_b = (int32_t)rows_b;
+    p.K = (int32_t)a.K;
+    p.ks_total = (int32_t)((a.K + BK - 1) / BK);
+    p.sf_col_tiles = (int32_t)((a.K / kb + 3) / 4);
+    p.sfa_row_tiles = (int32_t)((rows_a + 127) / 128);
+    p.sfb_row_tiles = (int32_t)((rows_b + 127) / 128);
+    p.alpha = a.alpha;
+    p.D = a.D;
+    p.ldd = a.ldd;
+    p.ws = nullptr;
+    p.units = 0;
+    p.max_seg = 0;
+}
+
+cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
+{
+    CUtensorMap ta, tb;
+    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PREFILL_BN)) {
+        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+        return cudaErrorInvalidValue;
+    }
+    Params p;
+    fill_common(p, a, a.M, a.N, a.sA, a.sB);
+    p.tiles_m = (int32_t)((a.M + BM - 1) / BM);
+    p.tiles_n = (int32_t)((a.N + PREFILL_BN - 1) / PREFILL_BN);
+    const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
+    const int grid = (int)(tiles < dev.sm_count ? tiles : dev.sm_count);
+    if (a.fmt == kMx)
+        return launch_kernel<PREFILL_BN, PREFILL_STAGES, true, false>(ta, tb, p, grid, s);
+    return launch_kernel<PREFILL_BN, PREFILL_STAGES, false, false>(ta, tb, p, grid, s);
+}
+
+cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
+{
+    // swap: the weight operand B [N x K] is the 128-row MMA side, the M <= 16
+    // tokens form the N = 16 side
+    CUtensorMap tw, tx;
+    if (!make_map(&tw, a.B, a.N, a.K / 2, BM) || !make_map(&tx, a.A, a.M, a.K / 2, DECODE_BN)) {
+        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+        return cudaErrorInvalidValue;
+    }
+    Params p;
+    fill_common(p, a, a.N, a.M, a.sB, a.sA);
+    p.tiles_m = (int32_t)((a.N + BM - 1) / BM);
+    p.tiles_n = 1;
+    p.units = p.tiles_m * p.ks_total;
+    const int G = p.units < dev.sm_count ? p.units : dev.sm_count;
+    p.max_seg = decode_max_seg(p.units, G, p.ks_total);
+    p.ws = static_cast<float*>(a.ws);
+    cudaError_t e;
+    if (a.fmt == kMx)
+        e = launch_kernel<DECODE_BN, DECODE_STAGES, true, true>(tw, tx, p, G, s);
+    else
+        e = launch_kernel<DECODE_BN, DECODE_STAGES, false, true>(tw, tx, p, G, s);
+    if (e != cudaSuccess) return e;
+    const int64_t total = a.N * a.M;
+    const int threads = 256;
+    splitk_reduce_kernel<DECODE_BN><<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(
+        p.ws, p.max_seg, p.units, G, p.ks_total, (int)a.N, (int)a.M, a.alpha, a.D, a.ldd);
+    return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_error_word(unsigned int* word)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(word, g_fp4_error_word, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*word) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_fp4_error_word, &zero, sizeof(unsigned int));
+    }
+    return e;
+}
+
+}  // namespace fp4

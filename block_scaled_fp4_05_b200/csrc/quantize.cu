@@ -1,0 +1,386 @@
+// Block quantizer kernels: BF16 -> E2M1 codes + per-block scales (NVFP4 /
+// MXFP4), the per-tensor amax for S_global, and alpha = gsA * gsB.
+//
+// Method: "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell",
+// "1. The Dual-Level Mathematical Formulation" (S_global, S_block,j, q_i) and
+// the emulation script of "End-to-End Implementation" (block amax, 1e-8
+// clamp, S = 2^ceil(log2(amax/6)), nearest E2M1 value); MXFP4 block size and
+// E8M0 scale from "MXFP4" / "Core Facts".
+//
+// The kernels are HBM-bound (2 B read, 0.5 + 1/k B written per element).
+// One CTA owns one 128-row x 4-block tile of the output, which is exactly one
+// 512-byte scale tile in the MMA layout, so the scale bytes are assembled in
+// shared memory and written as one coalesced 512-byte chunk.  Inputs are read
+// with 128-bit streaming loads, 8 BF16 per thread per load; the block amax is
+// an integer max over BF16 magnitude bits, combined across the 2 (k=16) or 4
+// (k=32) lanes of a block with warp shuffles.
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+#include <cfloat>
+
+#include "fp4_internal.h"
+
+namespace fp4 {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Largest BF16 magnitude (sign cleared, as an integer) of 8 packed values.
+__device__ __forceinline__ uint32_t absmax8(uint4 v)
+{
+    const uint32_t m = 0x7FFF7FFFu;
+    uint32_t a = __vmaxu2(v.x & m, v.y & m);
+    uint32_t b = __vmaxu2(v.z & m, v.w & m);
+    a = __vmaxu2(a, b);
+    return max(a & 0xFFFFu, a >> 16);
+}
+
+// Unsigned E4M3 round-to-nearest-even, saturating at 448.
+__device__ __forceinline__ uint32_t cvt_e4m3(float t)
+{
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+    return r & 0xFFu;
+}
+
+__device__ __forceinline__ float e4m3_value(uint32_t byte)
+{
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)byte));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Block scale from the block's BF16 magnitude bits.  Writes the multiplier
+// applied to the elements and returns the stored scale byte.
+template <int FMT>
+__device__ __forceinline__ uint32_t block_scale(uint32_t amax_bits, float gs, float denom,
+                                                float* inv)
+{
+    const float amax = __uint_as_float(amax_bits << 16);
+    if (FMT == kMx) {
+        // e = ceil(log2(max(amax, 1e-8) / 6)).  For amax = f * 2^E, f in
+        // [1, 2): e = E - 2 when f <= 1.5, else E - 1 (f > 1.5 <=> the 7-bit
+        // BF16 mantissa exceeds 64).
+        int e;
+        if (amax < 1e-8f) {
+            e = -29;
+        } else {
+            const int Eb = (int)((amax_bits >> 7) & 0xFF);
+            e = Eb - 129 + ((amax_bits & 0x7F) > 64 ? 1 : 0);
+        }
+        *inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+        return (uint32_t)(e + 127);
+    } else {
+        const float t = __fdiv_rn(amax, denom);
+        const uint32_t sb = cvt_e4m3(t);
+        const float eff = __fmul_rn(e4m3_value(sb), gs);
+        *inv = (eff == 0.0f) ? 0.0f : fminf(__frcp_rn(eff), FLT_MAX);
+        return sb;
+    }
+}
+
+// Eight BF16 values times `inv` (FP32 products), rounded to E2M1 with
+// round-to-nearest-even and saturation: 8 nibbles, element 0 in the lowest.
+// cvt...e2m1x2 puts its first source in the high nibble, its second in the
+// low nibble.
+__device__ __forceinline__ uint32_t quantize8(uint4 v, float inv)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __fmul_rn(__uint_as_float(w[i] << 16), inv);
+        f[2 * i + 1] = __fmul_rn(__uint_as_float(w[i] & 0xFFFF0000u), inv);
+    }
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]));
+    return out;
+}
+
+// ---------------------------------------------------------------------------
+// Rowwise: CTA tile = 128 rows x 4k columns -> one 512-byte scale tile.
+// grid = (cols / 4k, ceil(rows / 128)).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                        const float* __restrict__ gs_ptr)
+{
+    constexpr int KB = FMT == kMx ? 32 : 16;     // elements per block
+    constexpr int TILE_C = 4 * KB;               // columns per CTA
+    constexpr int CPR = TILE_C / 8;              // 16-byte chunks per row
+    constexpr int RPP = kThreads / CPR;          // rows per pass
+    constexpr int PASSES = 128 / RPP;
+    constexpr int CPB = KB / 8;                  // chunks per block
+
+    __shared__ __align__(16) uint8_t s_tile[512];
+
+    const int tid = threadIdx.x;
+    const int cc = tid % CPR;
+    const int rsub = tid / CPR;
+    const int64_t ct = blockIdx.x;
+    const int64_t rt = blockIdx.y;
+    const int64_t c0 = ct * TILE_C;
+    const int64_t r0 = rt * 128;
+    const int64_t nct = cols / TILE_C;
+
+    float gs = 1.0f, denom = 6.0f;
+    if (FMT == kNv) {
+        gs = __ldg(gs_ptr);
+        denom = __fmul_rn(6.0f, gs);
+    }
+
+    uint4 v[PASSES];
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+        const int64_t r = r0 + rsub + p * RPP;
+        if (r < rows)
+            v[p] = ld_stream(reinterpret_cast<const uint4*>(x + r * ld + c0) + cc);
+        else
+            v[p] = make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    uint32_t* out32 = reinterpret_cast<uint32_t*>(packed);
+    const int64_t row_words = cols / 8;  // 4-byte words per packed row
+#pragma unroll
+    for (int p = 0; p < PASSES; ++p) {
+        const int rl = rsub + p * RPP;
+        const int64_t r = r0 + rl;
+        uint32_t am = absmax8(v[p]);
+        if (CPB >= 2) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+        if (CPB >= 4) am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+        float inv;
+        const uint32_t sbyte = block_scale<FMT>(am, gs, denom, &inv);
+        const uint32_t q = quantize8(v[p], inv);
+        if (r < rows)
+            out32[r * row_words + c0 / 8 + cc] = q;
+        if (cc % CPB == 0)
+            s_tile[(rl % 32) * 16 + (rl / 32) * 4 + cc / CPB] = (r < rows) ? (uint8_t)sbyte : 0;
+    }
+    __syncthreads();
+    if (tid < 32) {
+        const uint4 t = reinterpret_cast<const uint4*>(s_tile)[tid];
+        reinterpret_cast<uint4*>(scales + (rt * nct + ct) * 512)[tid] = t;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Colwise: blocks run down the columns; output row c = input column c.
+// CTA tile = 4k input rows (the blocked direction) x 128 input columns (the
+// output rows) -> one 512-byte scale tile.  The BF16 tile is staged through
+// shared memory, each thread then quantizes whole blocks (one column, k
+// consecutive rows), and the packed output tile is staged again so that the
+// global writes are coalesced.  grid = (rows / 4k, ceil(cols / 128)).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+quantize_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                        const float* __restrict__ gs_ptr)
+{
+    constexpr int KB = FMT == kMx ? 32 : 16;
+    constexpr int TILE_K = 4 * KB;                       // input rows per CTA
+    constexpr int LOAD_PASSES = TILE_K * 16 / kThreads;  // 16 chunks of 8 per input row
+    constexpr int OUT_BYTES = TILE_K / 2;                // packed bytes per output row
+
+    __shared__ __align__(16) uint16_t s_in[TILE_K][128];
+    __shared__ __align__(16) uint8_t s_out[128][OUT_BYTES];
+    __shared__ __align__(16) uint8_t s_tile[512];
+
+    const int tid = threadIdx.x;
+    const int64_t kt = blockIdx.x;        // scale-column tile (blocked direction)
+    const int64_t ot = blockIdx.y;        // output row tile
+    const int64_t k0 = kt * TILE_K;
+    const int64_t oc0 = ot * 128;
+    const int64_t nct = rows / TILE_K;
+
+    float gs = 1.0f, denom = 6.0f;
+    if (FMT == kNv) {
+        gs = __ldg(gs_ptr);
+        denom = __fmul_rn(6.0f, gs);
+    }
+
+    // coalesced load of the TILE_K x 128 BF16 tile (zero past the last column)
+#pragma unroll
+    for (int p = 0; p < LOAD_PASSES; ++p) {
+        const int lr = tid / 16 + p * (kThreads / 16);
+        const int ch = tid % 16;
+        const int64_t c = oc0 + ch * 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (c < cols)
+            v = ld_stream(reinterpret_cast<const uint4*>(x + (k0 + lr) * ld + c));
+        *reinterpret_cast<uint4*>(&s_in[lr][ch * 8]) = v;
+    }
+    __syncthreads();
+
+    // each thread: 2 blocks (output row o, block b); a warp covers 32
+    // consecutive output rows of one block, so shared reads are conflict-free
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int task = tid + i * kThreads;
+        const int o = task % 128;
+        const int b = task / 128;
+        uint32_t w[KB / 2];
+        uint32_t am = 0;
+#pragma unroll
+        for (int j = 0; j < KB / 2; ++j) {
+            const uint32_t lo = s_in[b * KB + 2 * j][o];
+            const uint32_t hi = s_in[b * KB + 2 * j + 1][o];
+            w[j] = lo | (hi << 16);
+            am = max(am, max(lo & 0x7FFFu, hi & 0x7FFFu));
+        }
+        float inv;
+        const uint32_t sbyte = block_scale<FMT>(am, gs, denom, &inv);
+#pragma unroll
+        for (int j = 0; j < KB / 8; ++j) {
+            const uint4 v = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            *reinterpret_cast<uint32_t*>(&s_out[o][b * (KB / 2) + 4 * j]) = quantize8(v, inv);
+        }
+        const bool valid = (oc0 + o) < cols;
+        s_tile[(o % 32) * 16 + (o / 32) * 4 + b] = valid ? (uint8_t)sbyte : 0;
+    }
+    __syncthreads();
+
+    // packed rows: OUT_BYTES per output row, 16 bytes per thread
+    constexpr int CH_PER_ROW = OUT_BYTES / 16;
+    const int64_t out_row_bytes = rows / 2;
+#pragma unroll
+    for (int p = 0; p < (128 * CH_PER_ROW) / kThreads; ++p) {
+        const int idx = tid + p * kThreads;
+        const int o = idx / CH_PER_ROW;
+        const int ch = idx % CH_PER_ROW;
+        if (oc0 + o < cols) {
+            const uint4 t = *reinterpret_cast<const uint4*>(&s_out[o][ch * 16]);
+            *reinterpret_cast<uint4*>(packed + (oc0 + o) * out_row_bytes + k0 / 2 + ch * 16) = t;
+        }
+    }
+    if (tid < 32) {
+        const uint4 t = reinterpret_cast<const uint4*>(s_tile)[tid];
+        reinterpret_cast<uint4*>(scales + (ot * nct + kt) * 512)[tid] = t;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// amax over a BF16 matrix into a 32-bit word (BF16 magnitude bits), then
+// S_global = amax / 2688 (1 when amax == 0) in place.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads)
+amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+            unsigned int* __restrict__ word)
+{
+    const int64_t cpr = cols / 8;
+    const int64_t total = rows * cpr;
+    uint32_t m = 0;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    for (; i + 3 * stride < total; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t j = i + u * stride;
+            const int64_t r = j / cpr, c = j % cpr;
+            v[u] = ld_stream(reinterpret_cast<const uint4*>(x + r * ld) + c);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) m = max(m, absmax8(v[u]));
+    }
+    for (; i < total; i += stride) {
+        const int64_t r = i / cpr, c = i % cpr;
+        m = max(m, absmax8(ld_stream(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    __shared__ uint32_t s_m[kThreads / 32];
+    if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kThreads / 32; ++w) b = max(b, s_m[w]);
+        if (b) atomicMax(word, b);
+    }
+}
+
+__global__ void global_scale_finalize_kernel(float* gs)
+{
+    const unsigned int bits = *reinterpret_cast<unsigned int*>(gs);
+    const float amax = __uint_as_float(bits << 16);
+    *gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+}
+
+__global__ void alpha_kernel(const float* a, const float* b, float* out)
+{
+    *out = __fmul_rn(*a, *b);
+}
+
+}  // namespace
+
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float* gs_out,
+                        cudaStream_t s)
+{
+    cudaError_t e = cudaMemsetAsync(gs_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    const int64_t chunks = rows * (cols / 8);
+    if (chunks > 0) {
+        DeviceInfo dev;
+        e = device_info(&dev);
+        if (e != cudaSuccess) return e;
+        int64_t grid = (chunks + kThreads - 1) / kThreads;
+        const int64_t cap = (int64_t)dev.sm_count * 8;
+        if (grid > cap) grid = cap;
+        amax_kernel<<<(unsigned)grid, kThreads, 0, s>>>(x, rows, cols, ld,
+                                                       reinterpret_cast<unsigned int*>(gs_out));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    global_scale_finalize_kernel<<<1, 1, 0, s>>>(gs_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s)
+{
+    alpha_kernel<<<1, 1, 0, s>>>(gsA, gsB, alpha);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
+                            int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
+                            cudaStream_t s)
+{
+    if (rows == 0 || cols == 0) return cudaSuccess;
+    const int kb = block_size(fmt);
+    if (axis == 0) {
+        dim3 grid((unsigned)(cols / (4 * kb)), (unsigned)((rows + 127) / 128));
+        if (fmt == kNv)
+            quantize_rowwise_kernel<kNv><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+        else
+            quantize_rowwise_kernel<kMx><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+    } else {
+        dim3 grid((unsigned)(rows / (4 * kb)), (unsigned)((cols + 127) / 128));
+        if (fmt == kNv)
+            quantize_colwise_kernel<kNv><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+        else
+            quantize_colwise_kernel<kMx><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fp4

@@ -1,0 +1,199 @@
+"""Python binding of libfp4 (include/fp4.h): argument marshalling only.
+
+Every function here passes device pointers of torch CUDA tensors and the
+current torch stream to the C ABI; all arithmetic runs in the library's CUDA
+kernels.  There is no fallback: if ``libfp4.so`` is missing or a call fails,
+an exception is raised.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+NVFP4, MXFP4 = 0, 1
+ROWWISE, COLWISE = 0, 1
+GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE = 0, 1, 2
+
+FP4_OK = 0
+STATUS_NAMES = {
+    0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE",
+    3: "FP4_ERR_MISALIGNED", 4: "FP4_ERR_CUDA", 5: "FP4_ERR_TIMEOUT", 6: "FP4_ERR_NO_DEVICE",
+}
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfp4.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "fp4.h")
+
+
+class Fp4Error(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__("%s%s" % (STATUS_NAMES.get(status, "status %d" % status),
+                                   (": " + what) if what else ""))
+
+
+_lib = None
+
+
+def lib():
+    """Load libfp4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libfp4.so is missing; build it with "
+                               "`python -m block_scaled_fp4_05_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        c = ctypes
+        P, i64, sz, st = c.c_void_p, c.c_int64, c.c_size_t, c.c_void_p
+        L.fp4_abi_version.restype = c.c_int
+        L.fp4_abi_version.argtypes = []
+        L.fp4_status_string.restype = c.c_char_p
+        L.fp4_status_string.argtypes = [c.c_int]
+        L.fp4_last_error.restype = c.c_char_p
+        L.fp4_last_error.argtypes = []
+        L.fp4_packed_bytes.restype = sz
+        L.fp4_packed_bytes.argtypes = [i64, i64]
+        L.fp4_scale_bytes.restype = sz
+        L.fp4_scale_bytes.argtypes = [c.c_int, i64, i64]
+        L.fp4_compute_global_scale.restype = c.c_int
+        L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
+        L.fp4_quantize.restype = c.c_int
+        L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
+        L.fp4_alpha_from_global_scales.restype = c.c_int
+        L.fp4_alpha_from_global_scales.argtypes = [P, P, P, st]
+        L.fp4_gemm.restype = c.c_int
+        L.fp4_gemm.argtypes = [c.c_int, P, P, P, P, i64, i64, i64, P, P, i64, P, sz, st]
+        L.fp4_gemm_with_kernel.restype = c.c_int
+        L.fp4_gemm_with_kernel.argtypes = [c.c_int, P, P, P, P, i64, i64, i64, P, P, i64, P, sz,
+                                           c.c_int, st]
+        L.fp4_gemm_workspace_bytes.restype = sz
+        L.fp4_gemm_workspace_bytes.argtypes = [c.c_int, i64, i64, i64]
+        L.fp4_get_device_status.restype = c.c_int
+        L.fp4_get_device_status.argtypes = [st]
+        _lib = L
+    return _lib
+
+
+def declared_symbols():
+    """Names of the functions declared in include/fp4.h."""
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(fp4_\w+)\s*\(", text, re.M)))
+
+
+def _check(status, what=""):
+    if status != FP4_OK:
+        detail = lib().fp4_last_error().decode()
+        raise Fp4Error(status, what + (" (%s)" % detail if detail else ""))
+
+
+def _stream(stream=None):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _dptr(t, what):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % what)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ld(t):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def block_size(fmt):
+    return 32 if fmt == MXFP4 else 16
+
+
+def fp4_status_string(status):
+    return lib().fp4_status_string(int(status)).decode()
+
+
+def fp4_packed_bytes(rows, k):
+    return lib().fp4_packed_bytes(int(rows), int(k))
+
+
+def fp4_scale_bytes(fmt, rows, k):
+    return lib().fp4_scale_bytes(int(fmt), int(rows), int(k))
+
+
+def fp4_compute_global_scale(x, gs_out, stream=None):
+    """S_global of bf16 matrix x into gs_out (float32 CUDA tensor, 1 element)."""
+    assert x.dtype == torch.bfloat16 and gs_out.dtype == torch.float32
+    _check(lib().fp4_compute_global_scale(_dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                                          _dptr(gs_out, "gs_out"), _stream(stream)),
+           "fp4_compute_global_scale")
+
+
+def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):
+    assert x.dtype == torch.bfloat16
+    _check(lib().fp4_quantize(int(fmt), int(axis), _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                              _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
+                              _dptr(global_scale, "global_scale"), _stream(stream)),
+           "fp4_quantize")
+
+
+def fp4_alpha_from_global_scales(gsA, gsB, alpha_out, stream=None):
+    _check(lib().fp4_alpha_from_global_scales(_dptr(gsA, "gsA"), _dptr(gsB, "gsB"),
+                                              _dptr(alpha_out, "alpha_out"), _stream(stream)),
+           "fp4_alpha_from_global_scales")
+
+
+def fp4_gemm_workspace_bytes(fmt, M, N, K):
+    return lib().fp4_gemm_workspace_bytes(int(fmt), int(M), int(N), int(K))
+
+
+def fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace=None, kernel=GEMM_AUTO, stream=None):
+    """D[M x N] (bf16, row stride D.stride(0)) = alpha * A_hat @ B_hat^T."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().fp4_gemm_with_kernel(int(fmt), _dptr(A, "A"), _dptr(sA, "sA"), _dptr(B, "B"),
+                                      _dptr(sB, "sB"), int(M), int(N), int(K),
+                                      _dptr(alpha, "alpha"), _dptr(D, "D"), D.stride(0),
+                                      _dptr(workspace, "workspace"), ws_bytes, int(kernel),
+                                      _stream(stream)),
+           "fp4_gemm")
+
+
+def fp4_get_device_status(stream=None):
+    return lib().fp4_get_device_status(_stream(stream))
+
+
+# ---------------------------------------------------------------------------
+# Allocating conveniences (torch provides the memory; the library computes)
+# ---------------------------------------------------------------------------
+def quantize(x, fmt, axis=ROWWISE, global_scale=None, stream=None):
+    """Quantize bf16 CUDA matrix x; returns (packed uint8 [R x K/2], scales uint8)."""
+    rows, cols = x.shape
+    out_rows, K = (rows, cols) if axis == ROWWISE else (cols, rows)
+    packed = torch.empty((out_rows, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((fp4_scale_bytes(fmt, out_rows, K),), dtype=torch.uint8, device=x.device)
+    fp4_quantize(fmt, axis, x, packed, scales, global_scale, stream)
+    return packed, scales
+
+
+def global_scale(x, stream=None):
+    gs = torch.empty((1,), dtype=torch.float32, device=x.device)
+    fp4_compute_global_scale(x, gs, stream)
+    return gs
+
+
+def gemm(fmt, A, sA, B, sB, K, alpha=None, kernel=GEMM_AUTO, out=None, workspace=None, stream=None):
+    """D = alpha * A_hat @ B_hat^T for packed operands; allocates D (and the
+    decode workspace when it applies) unless given."""
+    M, N = A.shape[0], B.shape[0]
+    D = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=A.device)
+    if workspace is None and kernel != GEMM_PREFILL:
+        nb = fp4_gemm_workspace_bytes(fmt, M, N, K)
+        if nb:
+            workspace = torch.empty((nb,), dtype=torch.uint8, device=A.device)
+    fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace, kernel, stream)
+    return D

@@ -1,0 +1,201 @@
+/*
+ * fp4.h -- C ABI of libfp4: microscaling FP4 quantization (NVFP4, MXFP4) and
+ * the native W4A4 block-scaled GEMM on NVIDIA B200 (sm_100a).
+ *
+ * The operations come from these web pages (cited by title and section):
+ *  [NVFP4-Arch] "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell"
+ *     "1. The E2M1 Floating-Point Format", "2. Micro-Block Exponent Scaling:
+ *     E8M0 Format", "1. The Dual-Level Mathematical Formulation",
+ *     "2. Hardware-Managed Tensor Core Dot-Products".
+ *  [ia4pymes]   "NVIDIA NVFP4 quantization ..." - "The Physics of NVFP4:
+ *     Block-Wise Microscaling Quantization" (16-element blocks, 8-bit scale).
+ *  [MXFP4-BW]   "How Microscaling FP4 (MXFP4) Halves Memory Bandwidth in
+ *     Frontier Models Without Training Divergence" - "The Microscaling
+ *     Breakthrough: 32-Element Blocks", "Silicon Execution: Tensor Cores &
+ *     Register Fusing".
+ *  [MXFP4-kc]   "MXFP4" - "Core Facts" (E8M0 scale, block size 32).
+ *
+ * Conventions shared by every entry point
+ *  - All data pointers are CUDA device pointers owned by the caller; the
+ *    library never allocates or frees caller-visible memory.
+ *  - Every call validates its arguments on the host first.  A call that
+ *    returns anything but FP4_OK has launched nothing.  A call that returns
+ *    FP4_OK has queued its kernels on `stream` (asynchronous; the results are
+ *    ready once the stream reaches that point).  Nothing is printed, nothing
+ *    aborts the process.
+ *  - BF16 inputs are row-major with a leading dimension `ld` in elements
+ *    (ld >= the row length, ld % 8 == 0) and a 16-byte aligned base pointer.
+ *    Outputs must be 16-byte aligned.
+ *  - Inputs must be finite: NaN or infinity give unspecified output bytes
+ *    (never a fault or a hang).
+ *  - Packed FP4: two E2M1 codes per byte, the even index in the low nibble,
+ *    K-major rows of K/2 bytes.  Code = sign bit (bit 3) | exponent (bits 2-1)
+ *    | mantissa (bit 0); values {0, 0.5, 1, 1.5, 2, 3, 4, 6} with signed zero.
+ *  - Scales: one byte per block (E4M3 for NVFP4, E8M0 for MXFP4) stored in
+ *    512-byte tiles of 128 rows x 4 block-columns, tiles ordered with the
+ *    block-column tile fastest; inside a tile the byte of (row r, block c) is
+ *    at (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  This is the layout the
+ *    tensor core's block-scaled MMA reads.  Padding rows are written as 0.
+ */
+#ifndef FP4_H
+#define FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* fp4_stream_t;
+
+typedef enum {
+    /* 16-element blocks, unsigned E4M3 block scale, FP32 per-tensor scale
+     * S_global ([NVFP4-Arch] dual-level formulation; [ia4pymes]). */
+    FP4_NVFP4 = 0,
+    /* 32-element blocks, E8M0 power-of-two block scale ([MXFP4-kc],
+     * [MXFP4-BW] "32-Element Blocks"). */
+    FP4_MXFP4 = 1
+} fp4_format;
+
+typedef enum {
+    /* blocks run along each row (the row is the K dimension) */
+    FP4_ROWWISE = 0,
+    /* blocks run down each column; output row c is input column c, i.e. the
+     * quantized result is the transpose (the K-major form of the other GEMM
+     * operand) */
+    FP4_COLWISE = 1
+} fp4_axis;
+
+typedef enum {
+    FP4_OK = 0,
+    FP4_ERR_INVALID_ARG = 1,       /* bad enum, NULL pointer, ld < length, small workspace */
+    FP4_ERR_UNSUPPORTED_SHAPE = 2, /* a dimension breaks a divisibility rule */
+    FP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension not 16-byte aligned */
+    FP4_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
+    FP4_ERR_TIMEOUT = 5,           /* a kernel gave up on a bounded wait (see fp4_get_device_status) */
+    FP4_ERR_NO_DEVICE = 6          /* no usable sm_100 device */
+} fp4_status;
+
+typedef enum {
+    FP4_GEMM_AUTO = 0,    /* decode kernel when M <= 16 and the workspace suffices, else prefill */
+    FP4_GEMM_PREFILL = 1, /* persistent 128x256-tile tensor-core kernel */
+    FP4_GEMM_DECODE = 2   /* swap-AB, stream-K kernel for M <= 16 plus a split-K reduction */
+} fp4_gemm_kernel;
+
+/* Version of this ABI (incremented on any signature change). */
+int fp4_abi_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp4_status_string(fp4_status s);
+
+/* Detail of the most recent failing call on this host thread (which check or
+ * CUDA call failed), or "" if none; valid until the thread's next failing
+ * call. */
+const char* fp4_last_error(void);
+
+/* Bytes of packed FP4 data for `rows` rows of length k: rows * k / 2. */
+size_t fp4_packed_bytes(int64_t rows, int64_t k);
+
+/* Bytes of the tiled scale buffer for `rows` rows of length k in format
+ * `fmt`: ceil(rows/128) * ceil(k/blk/4) * 512 (blk = 16 or 32).  0 for an
+ * invalid format. */
+size_t fp4_scale_bytes(fp4_format fmt, int64_t rows, int64_t k);
+
+/*
+ * S_global of a BF16 matrix: amax over |x| divided by 6 * 448 = 2688 in FP32,
+ * or 1.0 if the matrix is all zero.  With this value the block that holds the
+ * tensor's largest magnitude gets the largest E4M3 block scale (448).
+ * [NVFP4-Arch] "1. The Dual-Level Mathematical Formulation", item 1 (a
+ * per-tensor scalar for the tensor's dynamic ceiling; FP32 is this library's
+ * reading of its precision).
+ *   in_bf16 : device, rows x cols, leading dimension ld (elements)
+ *   gs_out  : device, one float, written asynchronously
+ * Requires cols % 8 == 0.
+ */
+fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t cols,
+                                    int64_t ld, float* gs_out, fp4_stream_t stream);
+
+/*
+ * Block quantization BF16 -> E2M1 codes + one scale per block.
+ * [NVFP4-Arch] "1. The Dual-Level Mathematical Formulation" (S_block,j,
+ * q_i = Quantize_E2M1(x_i / (S_global * S_block,j))) and the emulation script
+ * in "End-to-End Implementation" (block amax, 1e-8 clamp, ceil(log2(amax/6))).
+ *
+ * Per block of k elements (k = 16 NVFP4, 32 MXFP4) with amax = max |x_i|:
+ *   MXFP4: e = ceil(log2(max(amax, 1e-8) / 6)); scale byte = e + 127;
+ *          v_i = x_i * 2^-e.
+ *   NVFP4: t = amax / (6 * gs) (FP32); scale byte = E4M3 round-to-nearest-
+ *          even of t, saturating at 448; eff = E4M3(byte) * gs (FP32);
+ *          v_i = x_i * RN(1/eff) (0 when eff == 0).
+ *   q_i  = E2M1 round-to-nearest-even of v_i, |v| >= 6 -> 6, sign of x_i kept.
+ *
+ *   axis = FP4_ROWWISE: blocks along each row of in[rows x cols];
+ *          packed_out is [rows x cols/2] bytes, scales_out covers rows x
+ *          cols/k scales.  Requires cols % (4k) == 0 (64 / 128).
+ *   axis = FP4_COLWISE: blocks down each column; packed_out is
+ *          [cols x rows/2] (the transpose), scales_out covers cols x rows/k.
+ *          Requires rows % (4k) == 0 and cols % 8 == 0.
+ *   global_scale: device pointer to S_global (NVFP4, required); ignored and
+ *          may be NULL for MXFP4.
+ *   Sizes of the outputs: fp4_packed_bytes / fp4_scale_bytes with the output
+ *   row count and the blocked length.
+ */
+fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int64_t rows,
+                        int64_t cols, int64_t ld, void* packed_out, void* scales_out,
+                        const float* global_scale, fp4_stream_t stream);
+
+/* alpha = gsA * gsB (FP32), the factor that restores both per-tensor scales
+ * after the block-scaled product (NVFP4).  All three are device pointers. */
+fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, float* alpha_out,
+                                        fp4_stream_t stream);
+
+/*
+ * D = alpha * A_hat * B_hat^T with BF16 output, where A_hat[m,k] = q * S_block
+ * of A's block and likewise for B.  The tensor core multiplies the E2M1 codes
+ * of each block pair, scales the partial product by the two block scales and
+ * accumulates in FP32 ([NVFP4-Arch] "2. Hardware-Managed Tensor Core
+ * Dot-Products"; [MXFP4-BW] "Silicon Execution"); the operands are never
+ * widened to 16 bits.  D = BF16_RNE(alpha * acc).
+ *   A : packed [M x K/2], sA its scales (M rows, K/k blocks), from fp4_quantize
+ *   B : packed [N x K/2], sB its scales (N rows)
+ *   alpha : device pointer to one float, or NULL for 1.0
+ *   D : BF16 [M x N], leading dimension ldd (elements, ldd >= N, ldd % 8 == 0)
+ *   workspace / ws_bytes : scratch for the decode kernel's split-K partials
+ *          (fp4_gemm_workspace_bytes); may be NULL / 0, then the prefill
+ *          kernel runs for every M.
+ * Requires K % 64 == 0 (NVFP4) or K % 128 == 0 (MXFP4) and N % 8 == 0.  M and
+ * N tails are handled inside the kernels.  M == 0 or N == 0 is a no-op;
+ * K == 0 writes zeros.
+ */
+fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B,
+                    const void* sB, int64_t M, int64_t N, int64_t K, const float* alpha,
+                    void* D, int64_t ldd, void* workspace, size_t ws_bytes,
+                    fp4_stream_t stream);
+
+/* Same as fp4_gemm with an explicit kernel choice.  FP4_GEMM_DECODE needs
+ * M <= 16 and a workspace of fp4_gemm_workspace_bytes bytes (else
+ * FP4_ERR_INVALID_ARG / FP4_ERR_UNSUPPORTED_SHAPE). */
+fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, const void* B,
+                                const void* sB, int64_t M, int64_t N, int64_t K,
+                                const float* alpha, void* D, int64_t ldd, void* workspace,
+                                size_t ws_bytes, fp4_gemm_kernel kernel, fp4_stream_t stream);
+
+/* Workspace bytes the decode kernel needs for this shape on the current
+ * device (0 when the decode kernel does not apply, i.e. M > 16). */
+size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K);
+
+/*
+ * Synchronizes `stream`, then reports and clears the device error word of the
+ * current device: FP4_ERR_TIMEOUT if a kernel of this library gave up on a
+ * bounded wait since the last call (its outputs are then unspecified), else
+ * FP4_OK; FP4_ERR_CUDA if the synchronization itself failed.
+ */
+fp4_status fp4_get_device_status(fp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4_H */

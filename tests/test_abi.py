@@ -1,0 +1,77 @@
+"""The C-ABI library loads and exports every function include/fp4.h declares;
+host-side checks and size helpers work without a GPU (no compute calls)."""
+import ctypes
+
+import pytest
+
+from block_scaled_fp4_05_b200 import fp4
+
+
+def test_library_exports_every_declared_symbol():
+    L = fp4.lib()
+    names = fp4.declared_symbols()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.fp4_abi_version() == 1
+
+
+def test_status_strings():
+    for code, name in fp4.STATUS_NAMES.items():
+        assert fp4.fp4_status_string(code) == name
+    assert fp4.fp4_status_string(99) == "FP4_ERR_UNKNOWN"
+
+
+def test_size_helpers_match_oracle_layout(orc):
+    for fmt in (fp4.NVFP4, fp4.MXFP4):
+        k = fp4.block_size(fmt)
+        for rows, K in [(1, 512), (128, 4096), (129, 8192), (28672, 8192), (3, 128)]:
+            assert fp4.fp4_packed_bytes(rows, K) == rows * K // 2
+            assert fp4.fp4_scale_bytes(fmt, rows, K) == orc.scale_bytes(rows, K // k)
+    assert fp4.fp4_scale_bytes(7, 128, 512) == 0
+    assert fp4.fp4_packed_bytes(0, 512) == 0
+
+
+P = ctypes.c_void_p
+A16 = P(1 << 20)       # 16-byte aligned dummy address (never dereferenced)
+A1 = P((1 << 20) + 1)  # misaligned
+
+
+@pytest.mark.parametrize("args,want", [
+    ((5, 0, A16, 128, 512, 512, A16, A16, A16, None), 1),      # bad format
+    ((0, 3, A16, 128, 512, 512, A16, A16, A16, None), 1),      # bad axis
+    ((0, 0, A16, 128, 512, 256, A16, A16, A16, None), 1),      # ld < cols
+    ((0, 0, A16, 128, 512, 512, A16, A16, None, None), 1),     # NVFP4 without S_global
+    ((0, 0, None, 128, 512, 512, A16, A16, A16, None), 1),     # NULL input
+    ((0, 0, A16, 128, 480, 480, A16, A16, A16, None), 2),      # cols % 64
+    ((1, 0, A16, 128, 192, 192, A16, A16, None, None), 2),     # cols % 128 (MX)
+    ((1, 1, A16, 96, 64, 64, A16, A16, None, None), 2),        # colwise rows % 128 (MX)
+    ((0, 0, A1, 128, 512, 512, A16, A16, A16, None), 3),       # misaligned input
+    ((0, 0, A16, 128, 512, 516, A16, A16, A16, None), 3),      # ld % 8
+    ((0, 0, A16, 0, 512, 512, None, None, None, None), 0),     # empty: no-op
+    ((0, 0, A16, 128, 512, 512, A16, A16, A16, None), 6),      # valid, but no device here
+])
+def test_quantize_host_checks_without_gpu(args, want):
+    import torch
+    if torch.cuda.is_available() and want == 6:
+        pytest.skip("a device is present")
+    assert fp4.lib().fp4_quantize(*args) == want
+
+
+def test_gemm_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    g = L.fp4_gemm_with_kernel
+    assert g(9, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 1
+    assert g(0, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 7, None) == 1
+    assert g(0, A16, A16, A16, A16, 16, 16, 96, None, A16, 16, None, 0, 0, None) == 2
+    assert g(1, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 2
+    assert g(0, A16, A16, A16, A16, 16, 12, 64, None, A16, 16, None, 0, 0, None) == 2
+    assert g(0, A16, A16, A16, A16, 16, 16, 64, None, A1, 16, None, 0, 0, None) == 3
+    assert g(0, A16, A16, A16, A16, 16, 16, 64, None, A16, 8, None, 0, 0, None) == 1
+    assert g(0, A16, A16, A16, A16, 0, 16, 64, None, A16, 16, None, 0, 0, None) == 0
+    if not torch.cuda.is_available():
+        assert g(0, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 6
+        assert L.fp4_compute_global_scale(A16, 4, 8, 8, A16, None) == 6
+    assert L.fp4_compute_global_scale(A16, 4, 12, 12, A16, None) == 2
+    assert L.fp4_alpha_from_global_scales(None, A16, A16, None) == 1

@@ -1,0 +1,187 @@
+"""GPU parity of the block-scaled GEMM kernels against the oracle (FP64
+product of the dequantized operands), within the stated tolerance.  Operands
+are quantized by the oracle and uploaded, so that the GEMM is tested on its
+own; the end-to-end tests quantize on the GPU as well."""
+import numpy as np
+import pytest
+import torch
+
+from block_scaled_fp4_05_b200 import fp4, synth
+from gpu_util import assert_gemm_close, bf16_dev_to_f64, to_dev_bf16, to_dev_f32, to_dev_u8
+
+pytestmark = pytest.mark.gpu
+FMTS = [fp4.NVFP4, fp4.MXFP4]
+
+
+def oracle_operands(orc, fmt, A_bits, B_bits):
+    gsA = orc.global_scale(A_bits) if fmt == fp4.NVFP4 else 1.0
+    gsB = orc.global_scale(B_bits) if fmt == fp4.NVFP4 else 1.0
+    pA, sA = orc.quantize(fmt, 0, A_bits, gs=gsA)
+    pB, sB = orc.quantize(fmt, 0, B_bits, gs=gsB)
+    alpha = float(np.float32(gsA) * np.float32(gsB))
+    return pA, sA, pB, sB, alpha
+
+
+def run_gpu_gemm(fmt, pA, sA, pB, sB, K, alpha, kernel, ldd_pad=0):
+    M, N = pA.shape[0], pB.shape[0]
+    D = torch.full((M, N + ldd_pad), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Dv = D[:, :N]
+    fp4.gemm(fmt, to_dev_u8(pA), to_dev_u8(sA), to_dev_u8(pB), to_dev_u8(sB), K,
+             alpha=to_dev_f32(alpha), kernel=kernel, out=Dv)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    if ldd_pad:
+        assert torch.isnan(D[:, N:].float()).all()
+    return bf16_dev_to_f64(Dv)
+
+
+def test_constant_operands_exact():
+    # A_hat = 1, B_hat = 0.5 -> D = 0.5 K exactly, no oracle involved
+    for fmt in FMTS:
+        k = fp4.block_size(fmt)
+        M, N, K = 200, 264, 1024
+        one = 0x38 if fmt == fp4.NVFP4 else 127
+        A = torch.full((M, K // 2), 0x22, dtype=torch.uint8, device="cuda")
+        B = torch.full((N, K // 2), 0x11, dtype=torch.uint8, device="cuda")
+        sA = torch.full((fp4.fp4_scale_bytes(fmt, M, K),), one, dtype=torch.uint8, device="cuda")
+        sB = torch.full((fp4.fp4_scale_bytes(fmt, N, K),), one, dtype=torch.uint8, device="cuda")
+        for kernel in (fp4.GEMM_PREFILL,):
+            D = fp4.gemm(fmt, A, sA, B, sB, K, kernel=kernel)
+            torch.cuda.synchronize()
+            assert torch.all(D.float() == 0.5 * K), (fmt, D.float().unique()[:8])
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_tiny_config(orc, fmt):
+    A, B = synth.tiny_nv()
+    pA, sA, pB, sB, alpha = oracle_operands(orc, fmt, A, B)
+    D_orc, S = orc.gemm(fmt, pA, sA, pB, sB, alpha=alpha)
+    D = run_gpu_gemm(fmt, pA, sA, pB, sB, 512, alpha, fp4.GEMM_PREFILL)
+    assert_gemm_close(D, D_orc, S, "tiny")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("MNK", [(1, 8, 128), (3, 24, 256), (129, 136, 384), (200, 264, 640),
+                                 (300, 520, 1024), (128, 256, 2048), (257, 512, 128)])
+def test_prefill_ragged_shapes(orc, fmt, MNK):
+    M, N, K = MNK
+    if K % (64 if fmt == fp4.NVFP4 else 128):
+        pytest.skip("K not supported by the format")
+    A = synth.normal_bf16(M, K, seed=31, outlier_factor=50.0)
+    B = synth.normal_bf16(N, K, seed=31, tensor_id=1, sigma=0.02)
+    pA, sA, pB, sB, alpha = oracle_operands(orc, fmt, A, B)
+    D_orc, S = orc.gemm(fmt, pA, sA, pB, sB, alpha=alpha)
+    D = run_gpu_gemm(fmt, pA, sA, pB, sB, K, alpha, fp4.GEMM_PREFILL, ldd_pad=8)
+    assert_gemm_close(D, D_orc, S, "prefill %s" % (MNK,))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("MNK", [(1, 256, 512), (4, 1000, 1024), (16, 1024, 8192), (7, 136, 384)])
+def test_decode_kernel_shapes(orc, fmt, MNK):
+    M, N, K = MNK
+    if K % (64 if fmt == fp4.NVFP4 else 128):
+        pytest.skip("K not supported by the format")
+    A = synth.normal_bf16(M, K, seed=32, outlier_factor=100.0)
+    W = synth.normal_bf16(N, K, seed=32, tensor_id=1, sigma=0.02)
+    pA, sA, pW, sW, alpha = oracle_operands(orc, fmt, A, W)
+    D_orc, S = orc.gemm(fmt, pA, sA, pW, sW, alpha=alpha)
+    D = run_gpu_gemm(fmt, pA, sA, pW, sW, K, alpha, fp4.GEMM_DECODE, ldd_pad=8)
+    assert_gemm_close(D, D_orc, S, "decode %s" % (MNK,))
+    D2 = run_gpu_gemm(fmt, pA, sA, pW, sW, K, alpha, fp4.GEMM_PREFILL)
+    assert_gemm_close(D2, D_orc, S, "prefill-on-decode-shape %s" % (MNK,))
+
+
+def test_k_zero_and_empty():
+    A = torch.empty((4, 0), dtype=torch.uint8, device="cuda")
+    B = torch.empty((8, 0), dtype=torch.uint8, device="cuda")
+    s = torch.zeros((512,), dtype=torch.uint8, device="cuda")
+    D = torch.full((4, 8), 7.0, dtype=torch.bfloat16, device="cuda")
+    fp4.fp4_gemm(fp4.NVFP4, A, s, B, s, 4, 8, 0, None, D)
+    torch.cuda.synchronize()
+    assert torch.all(D.float() == 0)
+    fp4.fp4_gemm(fp4.NVFP4, A, s, B, s, 0, 8, 64, None, D)   # M == 0: no-op
+
+
+def test_invalid_arguments_launch_nothing():
+    d = torch.zeros((1024,), dtype=torch.uint8, device="cuda")
+    D = torch.zeros((16, 16), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(fp4.Fp4Error) as e:
+        fp4.fp4_gemm(fp4.NVFP4, d, d, d, d, 16, 16, 96, None, D)   # K % 64
+    assert e.value.status == 2
+    with pytest.raises(fp4.Fp4Error) as e:
+        fp4.fp4_gemm(fp4.MXFP4, d, d, d, d, 16, 16, 64, None, D)   # K % 128
+    assert e.value.status == 2
+    with pytest.raises(fp4.Fp4Error) as e:
+        fp4.fp4_gemm(fp4.NVFP4, d[1:], d, d, d, 16, 16, 64, None, D)   # misaligned
+    assert e.value.status == 3
+    with pytest.raises(fp4.Fp4Error) as e:
+        fp4.fp4_gemm(fp4.NVFP4, d, d, d, d, 32, 16, 64, None, D, kernel=fp4.GEMM_DECODE)
+    assert e.value.status in (1, 2)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_end_to_end_gpu_quantize_then_gemm(orc, fmt):
+    A = synth.normal_bf16(333, 1024, seed=33, outlier_factor=50.0)
+    B = synth.normal_bf16(264, 1024, seed=33, tensor_id=1)
+    Ad, Bd = to_dev_bf16(A), to_dev_bf16(B)
+    if fmt == fp4.NVFP4:
+        gA, gB = fp4.global_scale(Ad), fp4.global_scale(Bd)
+        alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+        fp4.fp4_alpha_from_global_scales(gA, gB, alpha)
+    else:
+        gA = gB = alpha = None
+    pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, gA)
+    pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, gB)
+    D = fp4.gemm(fmt, pA, sA, pB, sB, 1024, alpha=alpha)
+    torch.cuda.synchronize()
+    pAo, sAo, pBo, sBo, alpha_o = oracle_operands(orc, fmt, A, B)
+    D_orc, S = orc.gemm(fmt, pAo, sAo, pBo, sBo, alpha=alpha_o)
+    assert_gemm_close(bf16_dev_to_f64(D), D_orc, S, "e2e")
+
+
+# --------------------------------------------------------------------------
+# full-size configurations, oracle on sampled output elements
+# --------------------------------------------------------------------------
+def sampled_check(orc, fmt, A_bits, B_bits, kernel, n_pairs=4096):
+    M, K = A_bits.shape
+    N = B_bits.shape[0]
+    Ad, Bd = to_dev_bf16(A_bits), to_dev_bf16(B_bits)
+    gsA = orc.global_scale(A_bits) if fmt == fp4.NVFP4 else 1.0
+    gsB = orc.global_scale(B_bits) if fmt == fp4.NVFP4 else 1.0
+    pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, to_dev_f32(gsA) if fmt == fp4.NVFP4 else None)
+    pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, to_dev_f32(gsB) if fmt == fp4.NVFP4 else None)
+    alpha = float(np.float32(gsA) * np.float32(gsB))
+    D = fp4.gemm(fmt, pA, sA, pB, sB, K, alpha=to_dev_f32(alpha), kernel=kernel)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    rng = np.random.default_rng(34)
+    ms = np.concatenate([rng.integers(0, M, n_pairs), [0, M - 1, M - 1, 0]])
+    ns = np.concatenate([rng.integers(0, N, n_pairs), [0, N - 1, 0, N - 1]])
+    # oracle operands from the oracle's own quantizer, on the sampled rows only
+    um, inv_m = np.unique(ms, return_inverse=True)
+    un, inv_n = np.unique(ns, return_inverse=True)
+    qA, sqA = orc.quantize(fmt, 0, np.ascontiguousarray(A_bits[um]), gs=gsA)
+    qB, sqB = orc.quantize(fmt, 0, np.ascontiguousarray(B_bits[un]), gs=gsB)
+    D_orc, S = orc.gemm_pairs(fmt, qA, sqA, qB, sqB, inv_m, inv_n, alpha=alpha)
+    D_gpu = bf16_dev_to_f64(D)[ms, ns]
+    assert_gemm_close(D_gpu, D_orc, S, "sampled")
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_square_4096_sampled(orc, fmt):
+    A, B = synth.square(4096)
+    sampled_check(orc, fmt, A, B, fp4.GEMM_PREFILL)
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_config_sampled(orc, M):
+    W = synth.decode_weight()
+    A = synth.decode_activation(M)
+    sampled_check(orc, fp4.NVFP4, A, W, fp4.GEMM_DECODE, n_pairs=2048)
+
+
+@pytest.mark.parametrize("shape", [(8192, 28672, 8192), (8192, 8192, 28672)])
+def test_prefill_config_sampled(orc, shape):
+    M, N, K = shape
+    A, W = synth.prefill(M, N, K)
+    sampled_check(orc, fp4.NVFP4, A, W, fp4.GEMM_PREFILL, n_pairs=1024)

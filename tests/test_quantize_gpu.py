@@ -1,0 +1,171 @@
+"""GPU parity of the quantizer kernels against the oracle: packed nibbles and
+scale bytes must be identical, output guard bands untouched, scale padding
+zero.  Runs the kernels through the C ABI (ctypes binding)."""
+import numpy as np
+import pytest
+import torch
+
+from block_scaled_fp4_05_b200 import fp4, synth
+from gpu_util import Guarded, to_dev_bf16, to_dev_f32
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [fp4.NVFP4, fp4.MXFP4]
+
+
+def gpu_quantize(fmt, axis, x_bits, gs):
+    rows, cols = x_bits.shape
+    out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
+    x = to_dev_bf16(x_bits)
+    packed = Guarded(out_rows * K // 2)
+    scales = Guarded(fp4.fp4_scale_bytes(fmt, out_rows, K), fill=0x5A)
+    gsd = to_dev_f32(gs) if fmt == fp4.NVFP4 else None
+    fp4.fp4_quantize(fmt, axis, x, packed.view, scales.view, gsd)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    assert packed.guards_intact() and scales.guards_intact()
+    return packed.view.cpu().numpy().reshape(out_rows, K // 2), scales.view.cpu().numpy()
+
+
+def check(orc, fmt, axis, x_bits, gs=None):
+    if gs is None:
+        gs = orc.global_scale(x_bits) if fmt == fp4.NVFP4 else 1.0
+    p_gpu, s_gpu = gpu_quantize(fmt, axis, x_bits, gs)
+    p_orc, s_orc = orc.quantize(fmt, axis, x_bits, gs=gs)
+    bad = np.argwhere(p_gpu != p_orc)
+    assert bad.size == 0, ("packed mismatch", bad[:4].tolist(), p_gpu[tuple(bad[0])], p_orc[tuple(bad[0])])
+    bad = np.nonzero(s_gpu != s_orc)[0]
+    assert bad.size == 0, ("scale mismatch", bad[:4].tolist(), s_gpu[bad[:4]], s_orc[bad[:4]])
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("axis", [fp4.ROWWISE, fp4.COLWISE])
+def test_tiny_config(orc, fmt, axis):
+    A, B = synth.tiny_nv()
+    check(orc, fmt, axis, A)
+    check(orc, fmt, axis, B)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(1, 512), (3, 256), (129, 384), (200, 1024), (517, 2048)])
+def test_rowwise_ragged_rows(orc, fmt, shape):
+    if shape[1] % (4 * fp4.block_size(fmt)):
+        pytest.skip("length not a multiple of 4 blocks")
+    x = synth.normal_bf16(*shape, seed=21, outlier_factor=60.0, zero_frac=0.05)
+    check(orc, fmt, fp4.ROWWISE, x)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(128, 8), (256, 24), (384, 136), (512, 1000)])
+def test_colwise_ragged_cols(orc, fmt, shape):
+    if shape[0] % (4 * fp4.block_size(fmt)):
+        pytest.skip("length not a multiple of 4 blocks")
+    x = synth.normal_bf16(*shape, seed=22, outlier_factor=60.0, zero_frac=0.05)
+    check(orc, fmt, fp4.COLWISE, x)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_all_zero_and_signed_zero(orc, fmt):
+    x = np.zeros((130, 256), dtype=np.uint16)
+    x[1::2, 5::3] = 0x8000  # -0.0
+    check(orc, fmt, fp4.ROWWISE, x, gs=1.0)
+    check(orc, fmt, fp4.COLWISE, np.zeros((256, 136), dtype=np.uint16), gs=1.0)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_rounding_ties_and_extremes(orc, fmt):
+    # blocks whose elements land exactly on the E2M1 decision points, plus
+    # the largest and smallest BF16 magnitudes and subnormals
+    rng = np.random.default_rng(23)
+    k = fp4.block_size(fmt)
+    ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 0.5, 1.0, 3.0, 4.0], dtype=np.float32)
+    rows = []
+    for e in range(-20, 21):
+        S = np.float32(2.0 ** e)
+        vals = np.resize(np.concatenate([ties, -ties]), k) * S
+        vals[0] = 6.0 * S   # amax = 6 S gives exponent e (MX)
+        rows.append(vals)
+    x = np.array(rows * 4, dtype=np.float32)
+    x = np.concatenate([x] * (128 // k), axis=1) if fmt == fp4.NVFP4 else np.concatenate([x] * 4, axis=1)
+    xb = synth.f32_to_bf16_bits(x)
+    extremes = np.array([0x7F7F, 0xFF7F, 0x0001, 0x8001, 0x0080, 0x007F, 0x3F80, 0xBF80],
+                        dtype=np.uint16)
+    xb[0, :8] = extremes
+    xb[1, :k] = rng.integers(1, 0x80, k).astype(np.uint16)  # subnormal block
+    check(orc, fmt, fp4.ROWWISE, xb, gs=1.0 if fmt == fp4.MXFP4 else 0.0625)
+    check(orc, fmt, fp4.ROWWISE, xb)
+
+
+def test_nv_custom_global_scales(orc):
+    x = synth.normal_bf16(256, 512, seed=24, outlier_factor=100.0)
+    for gs in [1.0, 2.0 ** -12, 0.0371, 1000.0]:
+        check(orc, fp4.NVFP4, fp4.ROWWISE, x, gs=gs)
+        check(orc, fp4.NVFP4, fp4.COLWISE, x, gs=gs)
+
+
+@pytest.mark.parametrize("shape", [(1, 8), (128, 512), (333, 4104), (4096, 4096)])
+def test_global_scale_matches_oracle(orc, shape):
+    x = synth.normal_bf16(*shape, seed=25, outlier_factor=50.0)
+    gs = fp4.global_scale(to_dev_bf16(x))
+    torch.cuda.synchronize()
+    assert np.float32(gs.item()) == np.float32(orc.global_scale(x))
+    z = fp4.global_scale(torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda"))
+    assert z.item() == 1.0
+
+
+def test_global_scale_with_leading_dimension(orc):
+    x = synth.normal_bf16(100, 256, seed=26, outlier_factor=10.0)
+    big = np.zeros((100, 512), dtype=np.uint16)
+    big[:, :256] = x
+    big[3, 300] = synth.f32_to_bf16_bits(np.array([1e6], dtype=np.float32))[0]  # outside the view
+    d = to_dev_bf16(big)
+    gs = fp4.global_scale(d[:, :256])
+    torch.cuda.synchronize()
+    assert np.float32(gs.item()) == np.float32(orc.global_scale(x))
+
+
+def test_alpha_from_global_scales():
+    a, b = to_dev_f32(0.0123), to_dev_f32(3.7)
+    out = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_alpha_from_global_scales(a, b, out)
+    torch.cuda.synchronize()
+    assert np.float32(out.item()) == np.float32(0.0123) * np.float32(3.7)
+
+
+# --------------------------------------------------------------------------
+# full-size sweep tensors (16384 x 16384 and 8192 x 28672): GPU output on
+# the whole tensor, oracle on a sample of output rows
+# --------------------------------------------------------------------------
+def sampled_rows_check(orc, fmt, axis, x_bits, n_rows=48):
+    rows, cols = x_bits.shape
+    gs = orc.global_scale(x_bits) if fmt == fp4.NVFP4 else 1.0
+    x = to_dev_bf16(x_bits)
+    packed, scales = fp4.quantize(x, fmt, axis, to_dev_f32(gs) if fmt == fp4.NVFP4 else None)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
+    rng = np.random.default_rng(27)
+    pick = np.unique(np.concatenate([[0, out_rows - 1], rng.integers(0, out_rows, n_rows)]))
+    if axis == fp4.ROWWISE:
+        sub = np.ascontiguousarray(x_bits[pick, :])
+        p_orc, _, rm = orc.quantize(fmt, fp4.ROWWISE, sub, gs=gs, with_rowmajor_scales=True)
+    else:
+        sub = np.ascontiguousarray(x_bits[:, pick])
+        p_orc, _, rm = orc.quantize(fmt, fp4.COLWISE, sub, gs=gs, with_rowmajor_scales=True)
+    p_gpu = packed[torch.from_numpy(pick).cuda()].cpu().numpy()
+    assert np.array_equal(p_gpu, p_orc)
+    s_all = scales.cpu().numpy()
+    nsc = K // fp4.block_size(fmt)
+    cols_idx = np.arange(nsc)
+    for i, r in enumerate(pick):
+        offs = [orc.scale_offset(int(r), int(c), nsc) for c in cols_idx]
+        assert np.array_equal(s_all[offs], rm[i])
+    return gs
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("axis", [fp4.ROWWISE, fp4.COLWISE])
+@pytest.mark.parametrize("shape", [(16384, 16384), (8192, 28672)])
+def test_full_size_sweep_sampled(orc, fmt, axis, shape):
+    x = synth.quant_sweep(*shape)
+    sampled_rows_check(orc, fmt, axis, x)
