@@ -1,0 +1,619 @@
+"""Benchmark of the block-scaled FP4 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one pass of the whole path over one batch of synthetic input.
+The default workload is the MXFP4 square case M = N = K = 4096: quantize A,
+quantize B (BF16 -> E2M1 + E8M0 block scales), then the block-scaled GEMM
+D = A_hat B_hat^T in BF16.  Other workloads (the decode, prefill and
+quantizer-sweep shapes) are selectable for measurement.
+
+Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs an
+independent replica (the path does not shard across GPUs: no data-path
+collective); NCCL is used only for the barrier and the max-over-ranks time.
+`--impl reference` times the CPU oracle (the reference implementation of
+the method in this repository) on a bounded sample of the same workload.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_scaled_fp4_05_b200 import fp4, synth  # noqa: E402
+
+METRIC = "FP4 GEMM TFLOPS & quantize GB/s on 1 B200; % of FP4 peak / HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_PER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput ratio (9 : 2.25 PFLOP/s)
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, traffic
+# ---------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index) \
+            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.strip()]
+        if self.path:
+            with open(self.path, "w") as f:
+                f.write(out)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("gemm.cu", "quantize.cu"):
+        with open(os.path.join(ROOT, "block_scaled_fp4_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            parts = line.split()
+            if len(parts) >= 4 and parts[0] == workload and parts[1] == kernel and parts[3] == want:
+                return float(parts[2])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+class Workload:
+    """Holds device buffers for R rotating input sets and the bound calls of
+    one step per set.  `kernels` names the timed kernel groups of a step."""
+    name = ""
+    unit = "TFLOP/s"
+
+    def step(self, i, ev=None):
+        calls = self.calls[i % len(self.calls)]
+        for k, group in enumerate(calls):
+            if ev is not None:
+                ev[k][0].record()
+            for c in group:
+                c()
+            if ev is not None:
+                ev[k][1].record()
+
+
+def _dev_bf16(bits, dev):
+    return synth.bits_to_torch(bits).to(dev)
+
+
+def _qbufs(fmt, rows, K, dev):
+    return (torch.empty((rows, K // 2), dtype=torch.uint8, device=dev),
+            torch.empty((fp4.fp4_scale_bytes(fmt, rows, K),), dtype=torch.uint8, device=dev))
+
+
+class SquareWorkload(Workload):
+    """Quantize A and B (rowwise, along K) and D = A_hat B_hat^T, M=N=K=n."""
+
+    def __init__(self, fmt, n, dev, sets=4):
+        self.fmt, self.n = fmt, n
+        self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
+        A, B = synth.square(n)
+        self.host = (A, B)
+        self.kernels = ["quantize_A", "quantize_B", "gemm"] if fmt == fp4.MXFP4 else \
+            ["global_scales", "quantize_A", "quantize_B", "gemm"]
+        self.calls = []
+        self.bufs = []
+        for s in range(sets):
+            Ad, Bd = _dev_bf16(A, dev), _dev_bf16(B, dev)
+            pA, sA = _qbufs(fmt, n, n, dev)
+            pB, sB = _qbufs(fmt, n, n, dev)
+            D = torch.empty((n, n), dtype=torch.bfloat16, device=dev)
+            groups = []
+            if fmt == fp4.NVFP4:
+                gA = torch.empty(1, dtype=torch.float32, device=dev)
+                gB = torch.empty(1, dtype=torch.float32, device=dev)
+                al = torch.empty(1, dtype=torch.float32, device=dev)
+                groups.append([fp4.bind_global_scale(Ad, gA), fp4.bind_global_scale(Bd, gB),
+                               fp4.bind_alpha(gA, gB, al)])
+            else:
+                gA = gB = al = None
+            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Ad, pA, sA, gA)])
+            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB)])
+            groups.append([fp4.bind_gemm(fmt, pA, sA, pB, sB, n, n, n, al, D, None, fp4.GEMM_PREFILL)])
+            self.calls.append(groups)
+            self.bufs.append((Ad, Bd, pA, sA, pB, sB, D, gA, gB, al))
+        kb = fp4.block_size(fmt)
+        qbytes = n * n * 2 + n * n // 2 + fp4.fp4_scale_bytes(fmt, n, n)
+        self.work = {"quantize_A": qbytes, "quantize_B": qbytes, "gemm": 2.0 * n ** 3,
+                     "global_scales": 2.0 * n * n * 2}
+        self.bound = {"quantize_A": "hbm", "quantize_B": "hbm", "gemm": "tensor",
+                      "global_scales": "hbm"}
+        self.flops = 2.0 * n ** 3
+        self.launches_per_step = 3 if fmt == fp4.MXFP4 else 3 + 2 * 2 + 1
+        self.dominant = "gemm"
+        self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
+            sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
+        del kb
+
+    def value(self, sec_per_step):
+        return self.flops / sec_per_step / 1e12
+
+    def e2e_setup(self, dev):
+        A, B = self.host
+        self.hA = synth.bits_to_torch(A).pin_memory()
+        self.hB = synth.bits_to_torch(B).pin_memory()
+        self.hD = torch.empty((self.n, self.n), dtype=torch.bfloat16).pin_memory()
+        return 2 * self.hA.numel() * 2, self.hD.numel() * 2
+
+    def e2e_step(self, dev):
+        fmt, n = self.fmt, self.n
+        Ad = self.hA.to(dev, non_blocking=True)
+        Bd = self.hB.to(dev, non_blocking=True)
+        if fmt == fp4.NVFP4:
+            gA, gB = fp4.global_scale(Ad), fp4.global_scale(Bd)
+            al = torch.empty(1, dtype=torch.float32, device=dev)
+            fp4.fp4_alpha_from_global_scales(gA, gB, al)
+        else:
+            gA = gB = al = None
+        pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, gA)
+        pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, gB)
+        D = fp4.gemm(fmt, pA, sA, pB, sB, n, alpha=al, kernel=fp4.GEMM_PREFILL)
+        self.hD.copy_(D, non_blocking=True)
+
+    def oracle_sample(self, orc, r):
+        """Oracle on an r x r sub-problem of the step: S_global passes (NVFP4)
+        and quantization of r rows of A and of B, then the FP64 GEMM of the
+        r x r output block; returns (extrapolated seconds per full step,
+        seconds spent).  The quantization uses the full tensors' S_global."""
+        A, B = self.host
+        n = self.n
+        fmt = orc.MXFP4 if self.fmt == fp4.MXFP4 else orc.NVFP4
+        if not hasattr(self, "_gs"):
+            self._gs = ((orc.global_scale(A), orc.global_scale(B)) if fmt == orc.NVFP4
+                        else (1.0, 1.0))
+        gsA, gsB = self._gs
+        a, b = np.ascontiguousarray(A[:r]), np.ascontiguousarray(B[:r])
+        t0 = time.perf_counter()
+        if fmt == orc.NVFP4:
+            orc.global_scale(a)
+            orc.global_scale(b)
+        pA, sA = orc.quantize(fmt, 0, a, gs=gsA)
+        pB, sB = orc.quantize(fmt, 0, b, gs=gsB)
+        t1 = time.perf_counter()
+        orc.gemm(fmt, pA, sA, pB, sB, alpha=float(np.float32(gsA) * np.float32(gsB)))
+        t2 = time.perf_counter()
+        return (t1 - t0) * (n / r) + (t2 - t1) * (n / r) ** 2, t2 - t0
+
+    def calibrate(self, orc, budget_s):
+        r = 32
+        while r < self.n:
+            _, spent = self.oracle_sample(orc, r)
+            if spent * 3.5 > budget_s:
+                break
+            r *= 2
+        return r
+
+    def cpu_baseline(self, orc, budget_s=20.0):
+        r = self.calibrate(orc, budget_s)
+        t_step, spent = self.oracle_sample(orc, r)
+        return {"value": self.flops / t_step / 1e12, "unit": "TFLOP/s",
+                "cores": orc.num_threads(), "kind": "oracle",
+                "sample": "S_global/quantization of %d rows of A and of B and the FP64 GEMM of "
+                          "the %dx%d output block (K=%d), extrapolated to the %dx%d step; "
+                          "%.1f s of CPU work in the measured sample"
+                          % (r, r, r, self.n, self.n, self.n, spent)}
+
+
+class DecodeWorkload(Workload):
+    """NVFP4 decode: W [28672 x 8192] quantized once; per step the M-token
+    activation gets S_global, is quantized, and D = A_hat W_hat^T runs on the
+    swap-AB stream-K kernel."""
+    unit = "GB/s"
+
+    def __init__(self, M, dev, sets=3, N=28672, K=8192):
+        self.M, self.N, self.K = M, N, K
+        self.name = "NVFP4 decode GEMM M=%d N=%d K=%d (W pre-quantized)" % (M, N, K)
+        W = synth.decode_weight(N, K)
+        A = synth.decode_activation(M, K)
+        self.host = (A, W)
+        self.kernels = ["act_global_scale", "act_quantize", "gemm"]
+        self.calls, self.bufs = [], []
+        Wd = _dev_bf16(W, dev)
+        gW = fp4.global_scale(Wd)
+        for s in range(sets):
+            pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
+            Ad = _dev_bf16(A, dev)
+            gA = torch.empty(1, dtype=torch.float32, device=dev)
+            al = torch.empty(1, dtype=torch.float32, device=dev)
+            pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
+            D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+            ws = torch.empty((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
+                             dtype=torch.uint8, device=dev)
+            self.calls.append([
+                [fp4.bind_global_scale(Ad, gA), fp4.bind_alpha(gA, gW, al)],
+                [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA)],
+                [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws, fp4.GEMM_DECODE)],
+            ])
+            self.bufs.append((pW, sW, Ad, gA, al, pA, sA, D, ws))
+        del Wd
+        torch.cuda.empty_cache()
+        wbytes = N * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, N, K)
+        abytes = M * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, M, K)
+        self.gemm_bytes = wbytes + abytes + M * N * 2
+        self.work = {"gemm": self.gemm_bytes, "act_quantize": M * K * 2 + abytes,
+                     "act_global_scale": M * K * 2}
+        self.bound = {"gemm": "hbm", "act_quantize": "hbm", "act_global_scale": "hbm"}
+        self.flops = 2.0 * M * N * K
+        self.launches_per_step = 2 + 1 + 1 + 2   # amax+finalize, alpha, quantize, gemm+reduce
+        self.dominant = "gemm"
+        self.l2_note = "rotating %d quantized weight copies (%.0f MB) > %d MB L2" % (
+            sets, sets * wbytes / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.gemm_bytes / sec_per_step / 1e9
+
+
+class QuantWorkload(Workload):
+    """One quantizer call on a sweep tensor (S_global given, computed once)."""
+    unit = "GB/s"
+
+    def __init__(self, fmt, axis, rows, cols, dev):
+        self.fmt, self.axis = fmt, axis
+        self.name = "%s %s quantize %dx%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4",
+                                              "rowwise" if axis == fp4.ROWWISE else "colwise",
+                                              rows, cols)
+        x = synth.quant_sweep(rows, cols)
+        self.host = (x,)
+        xd = _dev_bf16(x, dev)
+        gs = fp4.global_scale(xd) if fmt == fp4.NVFP4 else None
+        out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
+        p, s = _qbufs(fmt, out_rows, K, dev)
+        self.calls = [[[fp4.bind_quantize(fmt, axis, xd, p, s, gs)]]]
+        self.bufs = [(xd, gs, p, s)]
+        self.kernels = ["quantize"]
+        self.qbytes = rows * cols * 2 + out_rows * K // 2 + fp4.fp4_scale_bytes(fmt, out_rows, K)
+        self.work = {"quantize": self.qbytes}
+        self.bound = {"quantize": "hbm"}
+        self.flops = 0.0
+        self.launches_per_step = 1
+        self.dominant = "quantize"
+        self.l2_note = "input %.0f MB > %d MB L2" % (rows * cols * 2 / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.qbytes / sec_per_step / 1e9
+
+
+class PrefillWorkload(Workload):
+    """NVFP4 prefill: activation S_global + quantize per step, weights
+    quantized once, D = A_hat W_hat^T on the persistent tensor-core kernel."""
+
+    def __init__(self, M, N, K, dev):
+        self.M, self.N, self.K = M, N, K
+        self.name = "NVFP4 prefill GEMM M=%d N=%d K=%d" % (M, N, K)
+        A, W = synth.prefill(M, N, K)
+        self.host = (A, W)
+        Ad, Wd = _dev_bf16(A, dev), _dev_bf16(W, dev)
+        gW = fp4.global_scale(Wd)
+        pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
+        del Wd
+        gA = torch.empty(1, dtype=torch.float32, device=dev)
+        al = torch.empty(1, dtype=torch.float32, device=dev)
+        pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.calls = [[
+            [fp4.bind_global_scale(Ad, gA), fp4.bind_alpha(gA, gW, al)],
+            [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA)],
+            [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, None, fp4.GEMM_PREFILL)],
+        ]]
+        self.bufs = [(Ad, gA, al, pA, sA, pW, sW, D, gW)]
+        torch.cuda.empty_cache()
+        self.kernels = ["act_global_scale", "act_quantize", "gemm"]
+        abytes = M * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, M, K)
+        self.work = {"gemm": 2.0 * M * N * K, "act_quantize": M * K * 2 + abytes,
+                     "act_global_scale": M * K * 2}
+        self.bound = {"gemm": "tensor", "act_quantize": "hbm", "act_global_scale": "hbm"}
+        self.flops = 2.0 * M * N * K
+        self.launches_per_step = 2 + 1 + 1 + 1
+        self.dominant = "gemm"
+        self.l2_note = "operands %.0f MB > %d MB L2" % ((M + N) * K * 0.5625 / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.flops / sec_per_step / 1e12
+
+
+def make_workload(name, dev):
+    if name == "square_mx":
+        return SquareWorkload(fp4.MXFP4, 4096, dev)
+    if name == "square_nv":
+        return SquareWorkload(fp4.NVFP4, 4096, dev)
+    if name.startswith("decode_m"):
+        return DecodeWorkload(int(name[len("decode_m"):]), dev)
+    if name == "prefill_up":
+        return PrefillWorkload(8192, 28672, 8192, dev)
+    if name == "prefill_down":
+        return PrefillWorkload(8192, 8192, 28672, dev)
+    if name.startswith("quant_"):
+        _, shape, f, ax = name.split("_")
+        rows, cols = (16384, 16384) if shape == "16384" else (8192, 28672)
+        return QuantWorkload(fp4.NVFP4 if f == "nv" else fp4.MXFP4,
+                             fp4.ROWWISE if ax == "row" else fp4.COLWISE, rows, cols, dev)
+    raise SystemExit("unknown workload %r" % name)
+
+
+WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
+             "prefill_down"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
+                                for f in ("nv", "mx") for a in ("row", "col")]
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as orc
+    if args.workload != "square_mx" and args.workload != "square_nv":
+        raise SystemExit("the reference arm covers the square workloads")
+    fmt = fp4.MXFP4 if args.workload == "square_mx" else fp4.NVFP4
+
+    class HostOnly(SquareWorkload):
+        def __init__(self):
+            self.fmt, self.n = fmt, 4096
+            self.host = synth.square(4096)
+            self.flops = 2.0 * 4096 ** 3
+            self.name = "%s quantize+GEMM M=N=K=4096" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4")
+
+    wl = HostOnly()
+    # each step is a bounded sample: the whole run stays within a few minutes
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    r = wl.calibrate(orc, budget)
+    for _ in range(args.warmup):
+        wl.oracle_sample(orc, r)
+    secs = [wl.oracle_sample(orc, r)[0] for _ in range(args.steps)]
+    sec = statistics.median(secs)
+    v = wl.flops / sec / 1e12
+    sample = ("per step: S_global/quantization of %d rows of A and of B and the FP64 GEMM of "
+              "the %dx%d output block (K=4096), extrapolated to the 4096x4096 step" % (r, r, r))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.name},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": orc.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="square_mx", choices=WORKLOADS)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 3
+        if args.warmup is None:
+            args.warmup = 1
+        run_reference(args)
+        return
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    wl = make_workload(args.workload, dev)
+    per_step_guess = {"square_mx": 60e-6, "square_nv": 70e-6}.get(args.workload, 200e-6)
+    steps = args.steps if args.steps is not None else max(50, int(2.0 / per_step_guess))
+    warmup = args.warmup if args.warmup is not None else max(3, min(200, steps // 20))
+    stream = torch.cuda.current_stream()
+
+    for i in range(warmup):
+        wl.step(i)
+    torch.cuda.synchronize()
+    if fp4.fp4_get_device_status() != 0:
+        raise SystemExit("device status: a kernel timed out during warm-up")
+
+    # per-kernel events on a uniform sample of the timed steps
+    n_sample = min(steps, 256)
+    sample_every = max(1, steps // n_sample)
+    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+           for _ in wl.kernels] for _ in range(n_sample)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    j = 0
+    for i in range(steps):
+        if i % sample_every == 0 and j < n_sample:
+            wl.step(i, ev[j])
+            j += 1
+        else:
+            wl.step(i)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    status = fp4.fp4_get_device_status()
+    if status != 0:
+        raise SystemExit("device status: a kernel timed out in the timed region")
+
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    sec_per_step = elapsed_ms / 1e3 / steps
+    value = wl.value(sec_per_step) * world
+
+    kern_ms = {k: statistics.mean(e[ki][0].elapsed_time(e[ki][1]) for e in ev[:j])
+               for ki, k in enumerate(wl.kernels)}
+    peaks = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    rooflines = {}
+    for k in wl.kernels:
+        dur = kern_ms[k] / 1e3
+        if wl.bound[k] == "tensor":
+            ach = wl.work[k] / dur / 1e12
+            rooflines[k] = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
+                            "frac": ach / fp4_peak, "ms": kern_ms[k]}
+        else:
+            ach = wl.work[k] / dur / 1e9
+            rooflines[k] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": ach / peaks["hbm_gbs"], "ms": kern_ms[k]}
+    dom = dict(rooflines[wl.dominant])
+    dom.pop("ms")
+    dom["traffic"] = recorded_traffic(args.workload, wl.dominant)
+    dom["kernel"] = wl.dominant
+    dom["peak_source"] = ("%s: %s" % (peaks["source"],
+                                      "bf16 burst x %.0f (nominal FP4:BF16)" % FP4_PER_BF16
+                                      if dom["bound"] == "tensor" else "HBM copy"))
+
+    e2e = None
+    if not args.no_e2e and hasattr(wl, "e2e_setup"):
+        hb, db = wl.e2e_setup(dev)
+        for _ in range(3):
+            wl.e2e_step(dev)
+        torch.cuda.synchronize()
+        n_e2e = 20
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            wl.e2e_step(dev)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / n_e2e
+        if dist is not None:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": wl.value(e_ms / 1e3) * world, "unit": wl.unit, "h2d_bytes_per_step": hb,
+               "d2h_bytes_per_step": db, "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(wl, "cpu_baseline"):
+        import oracle as orc
+        cpu = wl.cpu_baseline(orc)
+
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": wl.unit, "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": sec_per_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e2m1 x e2m1 -> f32 accumulate, bf16 out",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "l2": wl.l2_note, "replicas": world,
+                   "inputs": "seeded synthetic BF16 (Philox), outlier channels"},
+        "roofline": dom,
+        "kernels": rooflines,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": wl.launches_per_step * steps,
+        "clocks": clk,
+    }
+    if args.workload.startswith("square"):
+        line["gemm_tflops"] = rooflines["gemm"]["achieved"]
+        line["quantize_gbs"] = statistics.mean(rooflines[k]["achieved"] for k in wl.kernels
+                                               if k.startswith("quantize"))
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

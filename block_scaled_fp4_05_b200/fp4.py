@@ -197,3 +197,43 @@ def gemm(fmt, A, sA, B, sB, K, alpha=None, kernel=GEMM_AUTO, out=None, workspace
             workspace = torch.empty((nb,), dtype=torch.uint8, device=A.device)
     fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace, kernel, stream)
     return D
+
+
+# ---------------------------------------------------------------------------
+# Pre-marshalled calls: the ctypes arguments are built once, each call then
+# costs one foreign call (used where launch overhead matters, e.g. decode).
+# ---------------------------------------------------------------------------
+class BoundCall:
+    def __init__(self, name, *cargs):
+        self._f = getattr(lib(), name)
+        self._args = cargs
+        self.name = name
+
+    def __call__(self):
+        st = self._f(*self._args)
+        if st != FP4_OK:
+            _check(st, self.name)
+
+
+def bind_global_scale(x, gs_out, stream=None):
+    return BoundCall("fp4_compute_global_scale", _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                     _dptr(gs_out, "gs_out"), _stream(stream))
+
+
+def bind_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):
+    return BoundCall("fp4_quantize", int(fmt), int(axis), _dptr(x, "x"), x.shape[0], x.shape[1],
+                     _ld(x), _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
+                     _dptr(global_scale, "global_scale"), _stream(stream))
+
+
+def bind_alpha(gsA, gsB, alpha_out, stream=None):
+    return BoundCall("fp4_alpha_from_global_scales", _dptr(gsA, "gsA"), _dptr(gsB, "gsB"),
+                     _dptr(alpha_out, "alpha_out"), _stream(stream))
+
+
+def bind_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace=None, kernel=GEMM_AUTO, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    return BoundCall("fp4_gemm_with_kernel", int(fmt), _dptr(A, "A"), _dptr(sA, "sA"),
+                     _dptr(B, "B"), _dptr(sB, "sB"), int(M), int(N), int(K),
+                     _dptr(alpha, "alpha"), _dptr(D, "D"), D.stride(0),
+                     _dptr(workspace, "workspace"), ws_bytes, int(kernel), _stream(stream))

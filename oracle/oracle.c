@@ -416,7 +416,7 @@ void orc_gemm(int fmt, const uint8_t* A, const uint8_t* sA, const uint8_t* B,
 {
     orc_dequantize(fmt, A, sA, M, K, 0.0, Adq);
     orc_dequantize(fmt, B, sB, N, K, 0.0, Bdq);
-    #pragma omp parallel for schedule(static)
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
             double acc = 0.0, mag = 0.0;
