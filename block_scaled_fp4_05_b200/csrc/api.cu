@@ -241,6 +241,35 @@ fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B
                                 FP4_GEMM_AUTO, stream);
 }
 
+fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA, const void* B,
+                                   const void* sB, int64_t M, int64_t N, int64_t K,
+                                   const float* alpha, void* D, int64_t ldd, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_fmt(fmt)) return FP4_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return FP4_ERR_INVALID_ARG;
+    if (M > 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0 || K == 0)   // nothing that needs scratch
+        return fp4_gemm_with_kernel(fmt, A, sA, B, sB, M, N, K, alpha, D, ldd, nullptr, 0,
+                                    FP4_GEMM_PREFILL, stream);
+    const size_t need = fp4_gemm_workspace_bytes(fmt, M, N, K);
+    if (need == 0) return FP4_ERR_NO_DEVICE;
+    if (need > fp4::noalloc_scratch_bytes()) {
+        snprintf(fp4::g_last_error, sizeof fp4::g_last_error,
+                 "decode partials need %zu bytes, above the %zu-byte static scratch", need,
+                 fp4::noalloc_scratch_bytes());
+        return FP4_ERR_UNSUPPORTED_SHAPE;
+    }
+    void* scratch = nullptr;
+    const cudaError_t e = fp4::noalloc_scratch(&scratch);
+    if (e != cudaSuccess) {
+        fp4::set_last_error("cudaGetSymbolAddress(static decode scratch)", e);
+        return from_cuda(e);
+    }
+    return fp4_gemm_with_kernel(fmt, A, sA, B, sB, M, N, K, alpha, D, ldd, scratch,
+                                fp4::noalloc_scratch_bytes(), FP4_GEMM_DECODE, stream);
+}
+
 fp4_status fp4_get_device_status(fp4_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

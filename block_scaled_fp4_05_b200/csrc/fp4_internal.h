@@ -48,6 +48,8 @@ size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
 cudaError_t read_and_clear_error_word(unsigned int* word);
+size_t noalloc_scratch_bytes();
+cudaError_t noalloc_scratch(void** out);
 int tensor_map_encoder_available();
 
 // Records the detail of a failure for fp4_last_error() (thread-local).

@@ -778,6 +778,42 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------------
+// Allocation-free decode: the split-K partials go to a fixed, file-scope
+// device array instead of a caller-provided workspace.  Every device that
+// loads the library holds these bytes until the process exits.  Successive
+// calls share the array and it keeps the last call's partials; nothing in it
+// needs to start at zero (each CTA writes every partial it later reads), but
+// two such calls that overlap on the GPU (different streams) race on it.
+// ------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of g_decode_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with that device current and cached.
+cudaError_t noalloc_scratch(void** out)
+{
+    static std::mutex mu;
+    static void* cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) {
+        *out = cache[dev];
+        return cudaSuccess;
+    }
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) cache[dev] = ptr;
+    *out = ptr;
+    return cudaSuccess;
+}
+
 cudaError_t read_and_clear_error_word(unsigned int* word)
 {
     cudaError_t e = cudaMemcpyFromSymbol(word, g_fp4_error_word, sizeof(unsigned int));

@@ -187,6 +187,37 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
 size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K);
 
 /*
+ * Allocation-free form of the decode GEMM (no counterpart on the pages: it is
+ * a service of this library, not part of the method).  Same operation,
+ * arguments, result and kernels as fp4_gemm_with_kernel(..., FP4_GEMM_DECODE),
+ * but the split-K partials live in a fixed 4 MiB array inside the library
+ * instead of a caller-provided workspace, and the call makes no device
+ * allocation of any kind.
+ *
+ * For callers that cannot call cudaMalloc on their hot path: plug-ins whose
+ * host framework owns the device's memory through its own pool (an allocation
+ * behind the pool's back escapes its accounting and fails once the pool has
+ * reserved the memory), and latency-bound loops where cudaMalloc/cudaFree
+ * would synchronize the device.
+ *
+ *  - Every GPU that loads the library holds the 4 MiB until the process exits.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the array and it keeps the last call's contents (nothing
+ *    in it has to start at zero).  Calls that overlap on the GPU (e.g. on two
+ *    streams at once) race on it: serialize them.
+ *  - Shapes whose partials exceed 4 MiB (fp4_gemm_workspace_bytes) are
+ *    rejected with FP4_ERR_UNSUPPORTED_SHAPE and an fp4_last_error() message;
+ *    M > 16 is rejected the same way.  (N = 28672, K = 8192 needs 3.6 MB on
+ *    148 SMs.)
+ */
+fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA, const void* B,
+                                   const void* sB, int64_t M, int64_t N, int64_t K,
+                                   const float* alpha, void* D, int64_t ldd,
+                                   fp4_stream_t stream);
+
+/*
  * Synchronizes `stream`, then reports and clears the device error word of the
  * current device: FP4_ERR_TIMEOUT if a kernel of this library gave up on a
  * bounded wait since the last call (its outputs are then unspecified), else
