@@ -12,22 +12,27 @@
 //   warp 0      TMA producer: packed A/B tiles via tensor maps (128-byte
 //               swizzle), scale chunks via 1-D bulk copies, into a ring of
 //               STAGES shared-memory stages guarded by full/empty mbarriers.
-//   warp 1      TMEM allocation; one thread issues tcgen05.cp (scales,
-//               shared -> tensor memory) and tcgen05.mma (kind::mxf4nvf4,
-//               block_scale, 128 x BN x 64 per instruction), then
-//               tcgen05.commit to release stages and to publish the
+//   warp 1      TMEM allocation; one thread issues tcgen05.mma
+//               (kind::mxf4nvf4, block_scale, 128 x BN x 64 per instruction)
+//               and tcgen05.commit to release stages and to publish the
 //               accumulator.
 //   warps 2-5   epilogue: tcgen05.ld of the FP32 accumulator (each warp its
-//               32-lane quadrant), alpha, BF16 round-to-nearest-even, 16-byte
-//               stores; or FP32 split-K partials (decode form).
+//               32-lane quadrant), alpha, BF16 round-to-nearest-even into
+//               registers, release of the accumulator, then 16-byte stores;
+//               or FP32 split-K partials (decode form).
+//   warps 6-9   scale staging: each warp copies the stage's scale chunks from
+//               shared memory into its own TMEM lane quadrant with
+//               tcgen05.st, so that the tensor pipe only runs MMAs (a
+//               tcgen05.cp of a 512-byte chunk occupies the tensor pipe for
+//               about half the time of a 128x256x64 MMA).
 // Every mbarrier wait is bounded by %globaltimer; on expiry the CTA sets the
 // library's device error word, stops issuing work, drains what it already
 // issued, frees its tensor memory and returns (no trap).
 //
 // Scale layout in tensor memory: one 512-byte chunk (128 rows x 4 scale
-// bytes, the global tile layout) is copied with tcgen05.cp 32x128b.warpx4 to
-// 4 TMEM columns; column c, lane l then holds the 4 scale bytes of row
-// 32c + l (replicated over the four lane quadrants).  For NVFP4
+// bytes, the global tile layout) occupies 4 TMEM columns; in every lane
+// quadrant, column c, lane l holds the 4 scale bytes of row 32c + l (lane l
+// of each staging warp writes the chunk's 16-byte row l).  For NVFP4
 // (scale_vec::4X, E4M3) one chunk serves one K=64 MMA; for MXFP4
 // (scale_vec::2X, E8M0) one chunk serves two, selected by scale-factor id 0/2.
 //
@@ -59,7 +64,7 @@ constexpr int MMA_K = 64;           // K per tcgen05.mma for FP4
 constexpr int A_BYTES = BM * BK_BYTES;
 constexpr int SF_CHUNK = 512;       // 128 rows x 4 scale bytes
 constexpr int SFA_BYTES = 4 * SF_CHUNK;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;    // 10 warps: producer, MMA, 4 epilogue, 4 scale staging
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum : unsigned { ERR_FULL = 1u, ERR_EMPTY = 2u, ERR_ACC_FULL = 4u, ERR_ACC_EMPTY = 8u,
@@ -79,9 +84,11 @@ struct Cfg {
     static constexpr int SFA_COLS = 4 * 4;               // 4 chunks x 4 columns
     static constexpr int SF_COLS = SFA_COLS + 4 * 4 * BH;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
     static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
+    static_assert(BH <= 2, "scale staging covers at most two 128-row tiles of B");
+    static_assert((3 * STAGES + 3) * 8 + 8 <= 512, "barrier area");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
 };
 
@@ -207,11 +214,6 @@ __device__ __forceinline__ void tc_commit(uint32_t bar)
                  : "memory");
 }
 
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc)
-{
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 template <bool MX>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
@@ -241,13 +243,6 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
 {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
            ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-// Descriptor of one 512-byte scale chunk: 32 rows of 16 bytes, no swizzle,
-// 8-row groups 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
-{
-    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(128 >> 4) << 32) | ((uint64_t)1 << 46);
 }
 
 // Instruction descriptor of kind::mxf4nvf4 with block scaling: E2M1 x E2M1,
@@ -281,6 +276,70 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16])
                    "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
                  :
                  : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+        " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32])
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                   "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                   "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                   "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                   "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                   "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32"
+        " [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32"
+        " [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
@@ -352,9 +411,9 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-    // bars[0..S): full, bars[S..2S): empty, bars[2S]: acc_full,
-    // bars[2S+1]: acc_empty, bars[2S+2]: drain
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 3);
+    // bars[0..S): full, [S..2S): empty, [2S..3S): scales staged,
+    // [3S]: acc_full, [3S+1]: acc_empty, [3S+2]: drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 3);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -362,14 +421,16 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     const uint32_t smem0 = smem_u32(smem);
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
-    const uint32_t acc_full = smem_u32(&bars[2 * STAGES]);
-    const uint32_t acc_empty = smem_u32(&bars[2 * STAGES + 1]);
-    const uint32_t drain = smem_u32(&bars[2 * STAGES + 2]);
+    auto sf_ready = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
+    const uint32_t acc_full = smem_u32(&bars[3 * STAGES]);
+    const uint32_t acc_empty = smem_u32(&bars[3 * STAGES + 1]);
+    const uint32_t drain = smem_u32(&bars[3 * STAGES + 2]);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full(s), 1);
             mbar_init(empty(s), 1);
+            mbar_init(sf_ready(s), 4);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4);
@@ -436,7 +497,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             }
             // Drain: the last min(issued, STAGES) stages may still be in flight
-            // if the consumer stopped early; wait for their transactions.
+            // if the consumers stopped early; wait for their transactions.
             if (!ok || *abort_flag) {
                 const int n = issued < STAGES ? issued : STAGES;
                 for (int i = 1; i <= n; ++i) {
@@ -461,28 +522,18 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             while (ok && sched.next(sg)) {
                 if (!wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
                 tc_fence_after();
-                const int rtb0 = (sg.tn * BN) / 128;
-                int nbh = 0;
-                for (int h = 0; h < C::BH; ++h)
-                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
                 for (int ks = sg.kb; ks < sg.ke; ++ks) {
-                    if (!wait_bounded(full(stage), phase, abort_flag, ERR_FULL)) {
+                    if (!wait_bounded(full(stage), phase, abort_flag, ERR_FULL) ||
+                        !wait_bounded(sf_ready(stage), phase, abort_flag, ERR_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int k0 = ks * BK;
                     const int nk = min(4, (p.K - k0) / MMA_K);
-                    const int nch = MX ? nk / 2 : nk;
                     const uint32_t st = smem0 + stage * C::STAGE_BYTES;
                     const uint32_t tsf = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
                     const uint32_t tsfb = tsf + C::SFA_COLS;
-                    for (int j = 0; j < nch; ++j) {
-                        tc_cp_sf(tsf + 4 * j, desc_sf(st + C::OFF_SFA + j * SF_CHUNK));
-                        for (int h = 0; h < nbh; ++h)
-                            tc_cp_sf(tsfb + (j * C::BH + h) * 4,
-                                     desc_sf(st + C::OFF_SFB + h * SFA_BYTES + j * SF_CHUNK));
-                    }
                     for (int j = 0; j < nk; ++j) {
                         const int chunk = MX ? (j >> 1) : j;
                         const uint32_t sf_id = MX ? (uint32_t)((j & 1) * 2) : 0u;
@@ -505,7 +556,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_commit(drain);
             wait_drain(drain, 0);
         }
-    } else {
+    } else if (warp < 6) {
         // ---------------- epilogue (warps 2..5) ----------------
         const int q = warp & 3;               // TMEM lane quadrant of this warp
         const int row = q * 32 + lane;        // accumulator row of this thread
@@ -523,34 +574,34 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             if (!ok) break;
             __syncwarp();
             tc_fence_after();
-            if (!STREAM_K) {
-                const int64_t gm = (int64_t)sg.tm * BM + row;
-                const bool row_ok = gm < p.rows_a;
-                uint16_t* drow = p.D + gm * p.ldd;
-#pragma unroll 1
-                for (int c = 0; c < BN / 16; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(trow + c * 16, r);
-                    tmem_wait_ld(r);
-                    const int gn0 = sg.tn * BN + c * 16;
-                    if (row_ok) {
+            if constexpr (!STREAM_K) {
+                // whole row of the tile into registers as BF16 pairs, then
+                // hand the accumulator back before the global stores
+                uint32_t packed[BN / 2];
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int gn = gn0 + 8 * h;
-                            if (gn < p.rows_b) {
-                                uint4 o;
-                                o.x = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 0])),
-                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 1])));
-                                o.y = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 2])),
-                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 3])));
-                                o.z = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 4])),
-                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 5])));
-                                o.w = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[8 * h + 6])),
-                                                  __fmul_rn(alpha, __uint_as_float(r[8 * h + 7])));
-                                *reinterpret_cast<uint4*>(drow + gn) = o;
-                            }
-                        }
-                    }
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(trow + c * 32, r);
+                    tmem_wait_ld(r);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        packed[c * 16 + i] =
+                            pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[2 * i])),
+                                        __fmul_rn(alpha, __uint_as_float(r[2 * i + 1])));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
+                const int64_t gm = (int64_t)sg.tm * BM + row;
+                if (gm < p.rows_a) {
+                    uint16_t* drow = p.D + gm * p.ldd + (int64_t)sg.tn * BN;
+                    const int ncols = p.rows_b - sg.tn * BN;
+#pragma unroll
+                    for (int i = 0; i < BN / 8; ++i)
+                        if (i * 8 < ncols)
+                            *reinterpret_cast<uint4*>(drow + i * 8) =
+                                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                           packed[4 * i + 3]);
                 }
             } else {
                 float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
@@ -563,11 +614,90 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     for (int j = 0; j < 16; ++j)
                         slot[(c * 16 + j) * BM + row] = __uint_as_float(r[j]);
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
             acc_phase ^= 1u;
+        }
+    } else {
+        // ---------------- scale staging (warps 6..9) ----------------
+        // Each warp writes its own TMEM lane quadrant: lane l stores the
+        // 16-byte row l of every 512-byte chunk (4 consecutive columns).
+        const uint32_t tq = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+        Schedule<STREAM_K> sched(p);
+        Seg sg;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        while (ok && sched.next(sg)) {
+            const int rtb0 = (sg.tn * BN) / 128;
+            int nbh = 0;
+            for (int h = 0; h < C::BH; ++h)
+                if (rtb0 + h < p.sfb_row_tiles) ++nbh;
+            for (int ks = sg.kb; ks < sg.ke; ++ks) {
+                int w = 0;
+                if (lane == 0) w = wait_bounded(full(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
+                w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                tc_fence_after();
+                const int k0 = ks * BK;
+                const int nk = min(4, (p.K - k0) / MMA_K);
+                const int nch = MX ? nk / 2 : nk;
+                const uint32_t st = smem0 + stage * C::STAGE_BYTES + lane * 16;
+                const uint32_t tsf = tq + C::SF_COL0 + stage * C::SF_COLS;
+                uint32_t a[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (j < nch) v = ld_shared_v4(st + C::OFF_SFA + j * SF_CHUNK);
+                    a[4 * j] = v.x;
+                    a[4 * j + 1] = v.y;
+                    a[4 * j + 2] = v.z;
+                    a[4 * j + 3] = v.w;
+                }
+                tmem_st16(tsf, a);
+                if constexpr (C::BH == 2) {
+                    uint32_t b[32];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (j < nch && h < nbh)
+                                v = ld_shared_v4(st + C::OFF_SFB + h * SFA_BYTES + j * SF_CHUNK);
+                            b[(j * 2 + h) * 4] = v.x;
+                            b[(j * 2 + h) * 4 + 1] = v.y;
+                            b[(j * 2 + h) * 4 + 2] = v.z;
+                            b[(j * 2 + h) * 4 + 3] = v.w;
+                        }
+                    tmem_st32(tsf + C::SFA_COLS, b);
+                } else {
+                    uint32_t b[16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (j < nch && nbh > 0) v = ld_shared_v4(st + C::OFF_SFB + j * SF_CHUNK);
+                        b[4 * j] = v.x;
+                        b[4 * j + 1] = v.y;
+                        b[4 * j + 2] = v.z;
+                        b[4 * j + 3] = v.w;
+                    }
+                    tmem_st16(tsf + C::SFA_COLS, b);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(sf_ready(stage));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
         }
     }
 
