@@ -173,6 +173,14 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Inline fast path: one try_wait, the bounded loop only when it fails.
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned code)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded(bar, parity, abort_flag, code);
+}
+
 // Wait that ignores the abort flag (used only to drain work already issued).
 __device__ __noinline__ bool wait_drain(uint32_t bar, uint32_t parity)
 {
@@ -456,6 +464,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            const uint32_t bar0 = smem_u32(bars);
+            const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
             Schedule<STREAM_K> sched(p);
             Seg sg;
             int stage = 0;
@@ -464,31 +474,32 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             bool ok = true;
             while (ok && sched.next(sg)) {
                 // scale row tiles of B that exist for this tile
-                int nbh = 0;
                 const int rtb0 = (sg.tn * BN) / 128;
+                int nbh = 0;
                 for (int h = 0; h < C::BH; ++h)
                     if (rtb0 + h < p.sfb_row_tiles) ++nbh;
+                const uint8_t* sfa_row = p.sfa + sg.tm * sf_row_bytes;
+                const uint8_t* sfb_row = p.sfb + rtb0 * sf_row_bytes;
+                const int ya = sg.tm * BM, yb = sg.tn * BN;
                 for (int ks = sg.kb; ks < sg.ke; ++ks) {
-                    if (!wait_bounded(empty(stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
+                    const uint32_t fb = bar0 + 8u * stage;
+                    if (!wait_fast(bar0 + 8u * (STAGES + stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
                         ok = false;
                         break;
                     }
-                    const int k0 = ks * BK;
-                    const int nk = min(4, (p.K - k0) / MMA_K);
+                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
                     const int nch = MX ? nk / 2 : nk;
-                    const int ct0 = MX ? k0 / 128 : k0 / 64;
+                    const int ct0 = MX ? ks * 2 : ks * 4;   // first 512-byte scale chunk of the stage
                     const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
                     const uint32_t st = smem0 + stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(full(stage), A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
-                    tma_load_2d(&tmA, full(stage), st, k0 / 2, sg.tm * BM);
-                    tma_load_2d(&tmB, full(stage), st + C::OFF_B, k0 / 2, sg.tn * BN);
-                    bulk_load(st + C::OFF_SFA,
-                              p.sfa + ((int64_t)sg.tm * p.sf_col_tiles + ct0) * SF_CHUNK, sf_bytes,
-                              full(stage));
-                    for (int h = 0; h < nbh; ++h)
-                        bulk_load(st + C::OFF_SFB + h * SFA_BYTES,
-                                  p.sfb + ((int64_t)(rtb0 + h) * p.sf_col_tiles + ct0) * SF_CHUNK,
-                                  sf_bytes, full(stage));
+                    mbar_arrive_expect_tx(fb, A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
+                    tma_load_2d(&tmA, fb, st, ks * BK_BYTES, ya);
+                    tma_load_2d(&tmB, fb, st + C::OFF_B, ks * BK_BYTES, yb);
+                    bulk_load(st + C::OFF_SFA, sfa_row + ct0 * SF_CHUNK, sf_bytes, fb);
+                    if (nbh > 0) bulk_load(st + C::OFF_SFB, sfb_row + ct0 * SF_CHUNK, sf_bytes, fb);
+                    if (C::BH == 2 && nbh > 1)
+                        bulk_load(st + C::OFF_SFB + SFA_BYTES, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
+                                  sf_bytes, fb);
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -513,36 +524,55 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
+        // The loop is kept short: a 128x256x64 MMA lasts 128 cycles, so the
+        // per-stage bookkeeping of this single thread must stay well below
+        // the 512 cycles of tensor work a 256-deep stage carries.
         if (lane == 0) {
+            const uint32_t bar0 = smem_u32(bars);
+            const uint64_t adesc0 = desc_sw128(smem0);
+            const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
+            constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;   // start-address field step
+            const uint32_t idesc0 = make_idesc<BN, MX>(0);
+            const uint32_t idesc2 = make_idesc<BN, MX>(2);
+            const uint32_t tsf0 = tmem_base + C::SF_COL0;
             Schedule<STREAM_K> sched(p);
             Seg sg;
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             while (ok && sched.next(sg)) {
-                if (!wait_bounded(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
+                if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
                 tc_fence_after();
                 for (int ks = sg.kb; ks < sg.ke; ++ks) {
-                    if (!wait_bounded(full(stage), phase, abort_flag, ERR_FULL) ||
-                        !wait_bounded(sf_ready(stage), phase, abort_flag, ERR_FULL)) {
+                    if (!wait_fast(bar0 + 8u * stage, phase, abort_flag, ERR_FULL) ||
+                        !wait_fast(bar0 + 8u * (2 * STAGES + stage), phase, abort_flag, ERR_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int k0 = ks * BK;
-                    const int nk = min(4, (p.K - k0) / MMA_K);
-                    const uint32_t st = smem0 + stage * C::STAGE_BYTES;
-                    const uint32_t tsf = tmem_base + C::SF_COL0 + stage * C::SF_COLS;
+                    const uint64_t ad = adesc0 + (uint64_t)(stage * kDescPerStage);
+                    const uint64_t bd = bdesc0 + (uint64_t)(stage * kDescPerStage);
+                    const uint32_t tsf = tsf0 + stage * C::SF_COLS;
                     const uint32_t tsfb = tsf + C::SFA_COLS;
-                    for (int j = 0; j < nk; ++j) {
-                        const int chunk = MX ? (j >> 1) : j;
-                        const uint32_t sf_id = MX ? (uint32_t)((j & 1) * 2) : 0u;
-                        const uint64_t ad = desc_sw128(st + j * 32);
-                        const uint64_t bd = desc_sw128(st + C::OFF_B + j * 32);
-                        tc_mma<MX>(tmem_base, ad, bd, make_idesc<BN, MX>(sf_id), tsf + 4 * chunk,
-                                   tsfb + chunk * C::BH * 4, (ks > sg.kb || j > 0) ? 1u : 0u);
+                    const uint32_t acc0 = ks > sg.kb ? 1u : 0u;
+                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                    if (nk == 4) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int chunk = MX ? (j >> 1) : j;
+                            tc_mma<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
+                                       (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
+                                       tsfb + chunk * C::BH * 4, j > 0 ? 1u : acc0);
+                        }
+                    } else {
+                        for (int j = 0; j < nk; ++j) {
+                            const int chunk = MX ? (j >> 1) : j;
+                            tc_mma<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
+                                       (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
+                                       tsfb + chunk * C::BH * 4, j > 0 ? 1u : acc0);
+                        }
                     }
-                    tc_commit(empty(stage));
+                    tc_commit(bar0 + 8u * (STAGES + stage));
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
