@@ -163,7 +163,7 @@ def _qbufs(fmt, rows, K, dev):
 class SquareWorkload(Workload):
     """Quantize A and B (rowwise, along K) and D = A_hat B_hat^T, M=N=K=n."""
 
-    def __init__(self, fmt, n, dev, sets=4):
+    def __init__(self, fmt, n, dev, sets=4, stream=None):
         self.fmt, self.n = fmt, n
         self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
         A, B = synth.square(n)
@@ -182,13 +182,14 @@ class SquareWorkload(Workload):
                 gA = torch.empty(1, dtype=torch.float32, device=dev)
                 gB = torch.empty(1, dtype=torch.float32, device=dev)
                 al = torch.empty(1, dtype=torch.float32, device=dev)
-                groups.append([fp4.bind_global_scale(Ad, gA), fp4.bind_global_scale(Bd, gB),
-                               fp4.bind_alpha(gA, gB, al)])
+                groups.append([fp4.bind_global_scale(Ad, gA, stream), fp4.bind_global_scale(Bd, gB, stream),
+                               fp4.bind_alpha(gA, gB, al, stream)])
             else:
                 gA = gB = al = None
-            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Ad, pA, sA, gA)])
-            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB)])
-            groups.append([fp4.bind_gemm(fmt, pA, sA, pB, sB, n, n, n, al, D, None, fp4.GEMM_PREFILL)])
+            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Ad, pA, sA, gA, stream)])
+            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB, stream)])
+            groups.append([fp4.bind_gemm(fmt, pA, sA, pB, sB, n, n, n, al, D, None, fp4.GEMM_PREFILL,
+                                         stream)])
             self.calls.append(groups)
             self.bufs.append((Ad, Bd, pA, sA, pB, sB, D, gA, gB, al))
         kb = fp4.block_size(fmt)
@@ -279,7 +280,7 @@ class DecodeWorkload(Workload):
     swap-AB stream-K kernel."""
     unit = "GB/s"
 
-    def __init__(self, M, dev, sets=3, N=28672, K=8192):
+    def __init__(self, M, dev, sets=3, N=28672, K=8192, stream=None):
         self.M, self.N, self.K = M, N, K
         self.name = "NVFP4 decode GEMM M=%d N=%d K=%d (W pre-quantized)" % (M, N, K)
         W = synth.decode_weight(N, K)
@@ -299,9 +300,9 @@ class DecodeWorkload(Workload):
             ws = torch.empty((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
                              dtype=torch.uint8, device=dev)
             self.calls.append([
-                [fp4.bind_global_scale(Ad, gA), fp4.bind_alpha(gA, gW, al)],
-                [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA)],
-                [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws, fp4.GEMM_DECODE)],
+                [fp4.bind_global_scale(Ad, gA, stream), fp4.bind_alpha(gA, gW, al, stream)],
+                [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA, stream)],
+                [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws, fp4.GEMM_DECODE, stream)],
             ])
             self.bufs.append((pW, sW, Ad, gA, al, pA, sA, D, ws))
         del Wd
@@ -326,7 +327,7 @@ class QuantWorkload(Workload):
     """One quantizer call on a sweep tensor (S_global given, computed once)."""
     unit = "GB/s"
 
-    def __init__(self, fmt, axis, rows, cols, dev):
+    def __init__(self, fmt, axis, rows, cols, dev, stream=None):
         self.fmt, self.axis = fmt, axis
         self.name = "%s %s quantize %dx%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4",
                                               "rowwise" if axis == fp4.ROWWISE else "colwise",
@@ -337,7 +338,7 @@ class QuantWorkload(Workload):
         gs = fp4.global_scale(xd) if fmt == fp4.NVFP4 else None
         out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
         p, s = _qbufs(fmt, out_rows, K, dev)
-        self.calls = [[[fp4.bind_quantize(fmt, axis, xd, p, s, gs)]]]
+        self.calls = [[[fp4.bind_quantize(fmt, axis, xd, p, s, gs, stream)]]]
         self.bufs = [(xd, gs, p, s)]
         self.kernels = ["quantize"]
         self.qbytes = rows * cols * 2 + out_rows * K // 2 + fp4.fp4_scale_bytes(fmt, out_rows, K)
@@ -356,7 +357,7 @@ class PrefillWorkload(Workload):
     """NVFP4 prefill: activation S_global + quantize per step, weights
     quantized once, D = A_hat W_hat^T on the persistent tensor-core kernel."""
 
-    def __init__(self, M, N, K, dev):
+    def __init__(self, M, N, K, dev, stream=None):
         self.M, self.N, self.K = M, N, K
         self.name = "NVFP4 prefill GEMM M=%d N=%d K=%d" % (M, N, K)
         A, W = synth.prefill(M, N, K)
@@ -370,9 +371,9 @@ class PrefillWorkload(Workload):
         pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
         D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         self.calls = [[
-            [fp4.bind_global_scale(Ad, gA), fp4.bind_alpha(gA, gW, al)],
-            [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA)],
-            [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, None, fp4.GEMM_PREFILL)],
+            [fp4.bind_global_scale(Ad, gA, stream), fp4.bind_alpha(gA, gW, al, stream)],
+            [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA, stream)],
+            [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, None, fp4.GEMM_PREFILL, stream)],
         ]]
         self.bufs = [(Ad, gA, al, pA, sA, pW, sW, D, gW)]
         torch.cuda.empty_cache()
@@ -390,22 +391,22 @@ class PrefillWorkload(Workload):
         return self.flops / sec_per_step / 1e12
 
 
-def make_workload(name, dev):
+def make_workload(name, dev, stream):
     if name == "square_mx":
-        return SquareWorkload(fp4.MXFP4, 4096, dev)
+        return SquareWorkload(fp4.MXFP4, 4096, dev, stream=stream)
     if name == "square_nv":
-        return SquareWorkload(fp4.NVFP4, 4096, dev)
+        return SquareWorkload(fp4.NVFP4, 4096, dev, stream=stream)
     if name.startswith("decode_m"):
-        return DecodeWorkload(int(name[len("decode_m"):]), dev)
+        return DecodeWorkload(int(name[len("decode_m"):]), dev, stream=stream)
     if name == "prefill_up":
-        return PrefillWorkload(8192, 28672, 8192, dev)
+        return PrefillWorkload(8192, 28672, 8192, dev, stream=stream)
     if name == "prefill_down":
-        return PrefillWorkload(8192, 8192, 28672, dev)
+        return PrefillWorkload(8192, 8192, 28672, dev, stream=stream)
     if name.startswith("quant_"):
         _, shape, f, ax = name.split("_")
         rows, cols = (16384, 16384) if shape == "16384" else (8192, 28672)
         return QuantWorkload(fp4.NVFP4 if f == "nv" else fp4.MXFP4,
-                             fp4.ROWWISE if ax == "row" else fp4.COLWISE, rows, cols, dev)
+                             fp4.ROWWISE if ax == "row" else fp4.COLWISE, rows, cols, dev, stream=stream)
     raise SystemExit("unknown workload %r" % name)
 
 
@@ -489,26 +490,51 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    wl = make_workload(args.workload, dev)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
+    wl = make_workload(args.workload, dev, stream)
     per_step_guess = {"square_mx": 60e-6, "square_nv": 70e-6}.get(args.workload, 200e-6)
     steps = args.steps if args.steps is not None else max(50, int(2.0 / per_step_guess))
     warmup = args.warmup if args.warmup is not None else max(3, min(200, steps // 20))
-    stream = torch.cuda.current_stream()
 
-    for i in range(warmup):
+    # eager warm-up (also sets every kernel's attributes before capture)
+    for i in range(max(3, len(wl.calls))):
         wl.step(i)
     torch.cuda.synchronize()
-    if fp4.fp4_get_device_status() != 0:
+    if fp4.fp4_get_device_status(stream) != 0:
         raise SystemExit("device status: a kernel timed out during warm-up")
 
-    # per-kernel events on a uniform sample of the timed steps
-    n_sample = min(steps, 256)
-    sample_every = max(1, steps // n_sample)
-    ev = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-           for _ in wl.kernels] for _ in range(n_sample)]
+    # The timed region replays CUDA graphs of the step (no host launch gaps):
+    # one graph of G consecutive steps (G a multiple of the rotating input
+    # sets), replayed steps // G times, plus a graph of the remainder.  In the
+    # last rotation of the G steps every kernel group is bracketed by timing
+    # events captured into the graph; the per-kernel times are those of the
+    # last replay.  (Events between every kernel would add gaps to the step.)
+    nsets = len(wl.calls)
+    G = min(steps, max(nsets, (32 // nsets) * nsets))
+    reps, rem = divmod(steps, G)
+    n_ev = min(G, nsets)
+    ev = [[[torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)] for _ in wl.kernels]
+          for _ in range(n_ev)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            e = G - 1 - i
+            wl.step(i, ev[e] if e < n_ev else None)
+    graph_rem = None
+    if rem:
+        graph_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_rem, stream=stream):
+            for i in range(rem):
+                wl.step(i)
+    for _ in range(max(1, warmup // G)):
+        graph.replay()
+    torch.cuda.synchronize()
+    warmup = max(3, nsets) + G * max(1, warmup // G)   # warm-up steps actually run
+
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -516,21 +542,19 @@ def main():
     clocks.start()
     time.sleep(0.3)
     t_start.record(stream)
-    j = 0
-    for i in range(steps):
-        if i % sample_every == 0 and j < n_sample:
-            wl.step(i, ev[j])
-            j += 1
-        else:
-            wl.step(i)
+    for _ in range(reps):
+        graph.replay()
+    if graph_rem is not None:
+        graph_rem.replay()
     t_end.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
-    status = fp4.fp4_get_device_status()
+    status = fp4.fp4_get_device_status(stream)
     if status != 0:
         raise SystemExit("device status: a kernel timed out in the timed region")
+    j = n_ev
 
     elapsed_ms = t_start.elapsed_time(t_end)
     if dist is not None:
@@ -589,6 +613,7 @@ def main():
         import oracle as orc
         cpu = wl.cpu_baseline(orc)
 
+    del graph, graph_rem
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

@@ -741,6 +741,444 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     }
 }
 
+// ------------------------------------------------------------------------
+// CTA-pair kernel (prefill).  A cluster of two CTAs on neighbouring SMs
+// computes a 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA stages
+// its own 128 rows of A and its half (128 rows) of the 256-row B tile, so a
+// CTA moves 32 KB of operands per 256-deep stage instead of 48 KB for the
+// same tensor work, and five stages fit in shared memory.  Each CTA keeps
+// the scales of its own A rows and of all 256 B rows in its own TMEM and
+// accumulates its 128 x 256 half of the tile there.
+//   - Both producers' A/B tensor loads complete on the leader's (rank 0)
+//     full[s] barrier; the leader's producer posts the expected bytes of
+//     both CTAs.  Scale chunks complete on each CTA's own sf_full[s].
+//   - Scale-staging warps of both CTAs arrive on the leader's sf_ready[s].
+//   - The leader's MMA thread issues the pair MMAs and releases stage s in
+//     both CTAs (and publishes the accumulator to both) with one commit
+//     that arrives on the barrier at the same offset in each CTA.
+//   - Epilogue warps of both CTAs arrive on the leader's acc_empty.
+// All waits are bounded; a CTA that gives up records the error, and both
+// CTAs meet at a final cluster barrier before the pair frees its TMEM.
+// ------------------------------------------------------------------------
+constexpr int PAIR_BN = 256;                 // N of the pair tile
+constexpr int PAIR_BHALF = PAIR_BN / 2;      // B rows staged by each CTA
+
+template <int STAGES>
+struct PairCfg {
+    static constexpr int B_BYTES = PAIR_BHALF * BK_BYTES;           // 16 KB
+    static constexpr int SFB_BYTES = 2 * SFA_BYTES;                 // 256 B rows: 2 row tiles
+    static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+    static constexpr int OFF_B = A_BYTES;
+    static constexpr int OFF_SFA = A_BYTES + B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    static constexpr int SF_COL0 = PAIR_BN;                        // accumulator: columns [0, 256)
+    static constexpr int SFA_COLS = 16;
+    static constexpr int SF_COLS = SFA_COLS + 32;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int NBARS = 5 * STAGES + 4;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 512;
+    static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
+    static_assert(NBARS * 8 + 8 <= 512, "barrier area");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// Arrive on a barrier of the other CTA without a cluster-scope release
+// fence.  Used only after tcgen05.wait::st, which already guarantees that the
+// tensor-memory writes the arrival announces have completed; the
+// cluster-scope release would cost ~1000 cycles per arrival.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+
+// 2-D tensor load whose completion is counted on a barrier of either CTA of
+// the pair (here: the leader's), destination in the issuing CTA.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster,
+                                                 uint32_t dst, int32_t x, int32_t y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+        : "memory");
+}
+
+// Arrive on the barrier at offset `bar` in both CTAs of the pair once the
+// pair MMAs issued so far have completed.
+__device__ __forceinline__ void tc_commit_pair_both(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)3)
+        : "memory");
+}
+
+template <bool MX>
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate)
+{
+    if (MX) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::2X"
+            " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+            " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    }
+}
+
+// Instruction descriptor of the pair MMA: M = 256 (128 rows per CTA), N = 256.
+template <bool MX>
+__device__ __forceinline__ uint32_t make_idesc_pair(uint32_t sf_id)
+{
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PAIR_BN >> 3) << 17) |
+           ((MX ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ void spin_ns(uint64_t ns)
+{
+    const uint64_t t0 = now_ns();
+    while (now_ns() - t0 < ns) {
+    }
+}
+
+template <int STAGES, bool MX>
+__global__ void __launch_bounds__(kThreads, 1)
+fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const Params p)
+{
+    using C = PairCfg<STAGES>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+    // [0,S) full (leader), [S,2S) empty, [2S,3S) sf_full, [3S,4S) sf_ready (leader),
+    // [4S] acc_full, [4S+1] acc_empty (leader), [4S+2] drain
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const uint32_t smem0 = smem_u32(smem);
+    const uint32_t bar0 = smem_u32(bars);
+    auto B_FULL = [&](int s) { return bar0 + 8u * s; };
+    auto B_EMPTY = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto B_SFFULL = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+    auto B_SFREADY = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
+    const uint32_t acc_full = bar0 + 8u * (4 * STAGES);
+    const uint32_t acc_empty = bar0 + 8u * (4 * STAGES + 1);
+    const uint32_t drain = bar0 + 8u * (4 * STAGES + 2);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(B_FULL(s), 1);
+            mbar_init(B_EMPTY(s), 1);
+            mbar_init(B_SFFULL(s), 1);
+            mbar_init(B_SFREADY(s), 8);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 8);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int tiles = p.tiles_m * p.tiles_n;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+            const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < tiles; t += npairs) {
+                const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+                const int rta = tm * 2 + (int)rank;                // this CTA's 128-row A tile
+                const bool has_sfa = rta < p.sfa_row_tiles;
+                int nbh = 0;
+                for (int h = 0; h < 2; ++h)
+                    if (tn * 2 + h < p.sfb_row_tiles) ++nbh;
+                const uint8_t* sfa_row = p.sfa + rta * sf_row_bytes;
+                const uint8_t* sfb_row = p.sfb + (int64_t)(tn * 2) * sf_row_bytes;
+                const int ya = rta * BM;
+                const int yb = tn * PAIR_BN + (int)rank * PAIR_BHALF;
+                for (int ks = 0; ks < p.ks_total; ++ks) {
+                    if (!wait_fast(B_EMPTY(stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                    const int nch = MX ? nk / 2 : nk;
+                    const int ct0 = MX ? ks * 2 : ks * 4;
+                    const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
+                    const uint32_t st = smem0 + stage * C::STAGE_BYTES;
+                    if (leader)
+                        mbar_arrive_expect_tx(B_FULL(stage), 2u * (A_BYTES + C::B_BYTES));
+                    const uint32_t full_leader = map_to_rank(B_FULL(stage), 0);
+                    tma_load_2d_pair(&tmA, full_leader, st, ks * BK_BYTES, ya);
+                    tma_load_2d_pair(&tmB, full_leader, st + C::OFF_B, ks * BK_BYTES, yb);
+                    mbar_arrive_expect_tx(B_SFFULL(stage), sf_bytes * ((has_sfa ? 1 : 0) + nbh));
+                    if (has_sfa)
+                        bulk_load(st + C::OFF_SFA, sfa_row + ct0 * SF_CHUNK, sf_bytes, B_SFFULL(stage));
+                    if (nbh > 0)
+                        bulk_load(st + C::OFF_SFB, sfb_row + ct0 * SF_CHUNK, sf_bytes, B_SFFULL(stage));
+                    if (nbh > 1)
+                        bulk_load(st + C::OFF_SFB + SFA_BYTES, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
+                                  sf_bytes, B_SFFULL(stage));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // On a give-up, give loads already issued time to land before the
+            // CTAs meet at the final cluster barrier.
+            if (!ok || *abort_flag) spin_ns(200000);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (leader CTA only) ----------------
+        if (lane == 0 && leader) {
+            const uint64_t adesc0 = desc_sw128(smem0);
+            const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
+            constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;
+            const uint32_t idesc0 = make_idesc_pair<MX>(0);
+            const uint32_t idesc2 = make_idesc_pair<MX>(2);
+            const uint32_t tsf0 = tmem_base + C::SF_COL0;
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; ok && t < tiles; t += npairs) {
+                if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
+                tc_fence_after();
+                for (int ks = 0; ks < p.ks_total; ++ks) {
+                    if (!wait_fast(B_FULL(stage), phase, abort_flag, ERR_FULL) ||
+                        !wait_fast(B_SFREADY(stage), phase, abort_flag, ERR_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = adesc0 + (uint64_t)(stage * kDescPerStage);
+                    const uint64_t bd = bdesc0 + (uint64_t)(stage * kDescPerStage);
+                    const uint32_t tsf = tsf0 + stage * C::SF_COLS;
+                    const uint32_t tsfb = tsf + C::SFA_COLS;
+                    const uint32_t acc0 = ks > 0 ? 1u : 0u;
+                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                    if (nk == 4) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int chunk = MX ? (j >> 1) : j;
+                            tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
+                                            (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
+                                            tsfb + chunk * 8, j > 0 ? 1u : acc0);
+                        }
+                    } else {
+                        for (int j = 0; j < nk; ++j) {
+                            const int chunk = MX ? (j >> 1) : j;
+                            tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
+                                            (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
+                                            tsfb + chunk * 8, j > 0 ? 1u : acc0);
+                        }
+                    }
+                    tc_commit_pair_both(B_EMPTY(stage));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair_both(acc_full);
+                acc_phase ^= 1u;
+            }
+            // every pair MMA issued here has completed before the TMEM is freed
+            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                             drain)
+                         : "memory");
+            wait_drain(drain, 0);
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue (warps 2..5, both CTAs) ----------------
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+        const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
+        uint32_t acc_phase = 0;
+        for (int t = pair; t < tiles; t += npairs) {
+            int ok = 0;
+            if (lane == 0) ok = wait_bounded(acc_full, acc_phase, abort_flag, ERR_ACC_FULL) ? 1 : 0;
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            if (!ok) break;
+            __syncwarp();
+            tc_fence_after();
+            uint32_t packed[PAIR_BN / 2];
+#pragma unroll
+            for (int c = 0; c < PAIR_BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld32(trow + c * 32, r);
+                tmem_wait_ld(r);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    packed[c * 16 + i] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[2 * i])),
+                                                     __fmul_rn(alpha, __uint_as_float(r[2 * i + 1])));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                if (leader)
+                    mbar_arrive(acc_empty);
+                else
+                    mbar_arrive_cluster_relaxed(acc_empty_leader);
+            }
+            const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+            const int64_t gm = (int64_t)(tm * 2 + (int)rank) * BM + row;
+            if (gm < p.rows_a) {
+                uint16_t* drow = p.D + gm * p.ldd + (int64_t)tn * PAIR_BN;
+                const int ncols = p.rows_b - tn * PAIR_BN;
+#pragma unroll
+                for (int i = 0; i < PAIR_BN / 8; ++i)
+                    if (i * 8 < ncols)
+                        *reinterpret_cast<uint4*>(drow + i * 8) =
+                            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
+                                       packed[4 * i + 3]);
+            }
+            acc_phase ^= 1u;
+        }
+    } else {
+        // ---------------- scale staging (warps 6..9, both CTAs) ----------------
+        const uint32_t tq = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = pair; ok && t < tiles; t += npairs) {
+            const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+            const bool has_sfa = tm * 2 + (int)rank < p.sfa_row_tiles;
+            int nbh = 0;
+            for (int h = 0; h < 2; ++h)
+                if (tn * 2 + h < p.sfb_row_tiles) ++nbh;
+            for (int ks = 0; ks < p.ks_total; ++ks) {
+                int w = 0;
+                if (lane == 0) w = wait_fast(B_SFFULL(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
+                w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                tc_fence_after();
+                const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                const int nch = MX ? nk / 2 : nk;
+                const uint32_t st = smem0 + stage * C::STAGE_BYTES + lane * 16;
+                const uint32_t tsf = tq + C::SF_COL0 + stage * C::SF_COLS;
+                uint32_t a[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (j < nch && has_sfa) v = ld_shared_v4(st + C::OFF_SFA + j * SF_CHUNK);
+                    a[4 * j] = v.x;
+                    a[4 * j + 1] = v.y;
+                    a[4 * j + 2] = v.z;
+                    a[4 * j + 3] = v.w;
+                }
+                tmem_st16(tsf, a);
+                uint32_t b[32];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (j < nch && h < nbh)
+                            v = ld_shared_v4(st + C::OFF_SFB + h * SFA_BYTES + j * SF_CHUNK);
+                        b[(j * 2 + h) * 4] = v.x;
+                        b[(j * 2 + h) * 4 + 1] = v.y;
+                        b[(j * 2 + h) * 4 + 2] = v.z;
+                        b[(j * 2 + h) * 4 + 3] = v.w;
+                    }
+                tmem_st32(tsf + C::SFA_COLS, b);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(B_SFREADY(stage));
+                    else
+                        mbar_arrive_cluster_relaxed(map_to_rank(B_SFREADY(stage), 0));
+                }
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();   // all pair MMAs done, both epilogues finished reading TMEM
+    tc_fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
 // Sum of the stream-K partials of each output element in CTA order, times
 // alpha, to BF16.  Output D[m][n] (m < tokens, n < weight rows).
 template <int BN>
@@ -890,22 +1328,63 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.max_seg = 0;
 }
 
+template <int STAGES, bool MX>
+cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
+                               int grid, cudaStream_t s)
+{
+    using C = PairCfg<STAGES>;
+    auto kern = fp4_gemm_pair_kernel<STAGES, MX>;
+    static std::mutex mu;
+    static uint64_t done_mask = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!(dev < 64 && ((done_mask >> dev) & 1ull))) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            if (e != cudaSuccess) {
+                set_last_error("cudaFuncSetAttribute(pair kernel)", e);
+                return e;
+            }
+            if (dev < 64) done_mask |= 1ull << dev;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+    if (e != cudaSuccess) set_last_error("pair GEMM kernel launch", e);
+    return e;
+}
+
+constexpr int PAIR_STAGES = 5;
+
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
 {
     CUtensorMap ta, tb;
-    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PREFILL_BN)) {
+    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PAIR_BHALF)) {
         set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return cudaErrorInvalidValue;
     }
     Params p;
     fill_common(p, a, a.M, a.N, a.sA, a.sB);
-    p.tiles_m = (int32_t)((a.M + BM - 1) / BM);
-    p.tiles_n = (int32_t)((a.N + PREFILL_BN - 1) / PREFILL_BN);
+    p.tiles_m = (int32_t)((a.M + 255) / 256);
+    p.tiles_n = (int32_t)((a.N + PAIR_BN - 1) / PAIR_BN);
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
-    const int grid = (int)(tiles < dev.sm_count ? tiles : dev.sm_count);
-    if (a.fmt == kMx)
-        return launch_kernel<PREFILL_BN, PREFILL_STAGES, true, false>(ta, tb, p, grid, s);
-    return launch_kernel<PREFILL_BN, PREFILL_STAGES, false, false>(ta, tb, p, grid, s);
+    const int64_t max_pairs = dev.sm_count / 2;
+    const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
+    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES, true>(ta, tb, p, grid, s);
+    return launch_pair_kernel<PAIR_STAGES, false>(ta, tb, p, grid, s);
 }
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
