@@ -131,6 +131,21 @@ def recorded_traffic(workload, kernel):
     return None
 
 
+def max_over_ranks(value, dist=None, device=None):
+    """Largest value over all ranks (the job's time is its slowest rank's)."""
+    if dist is None:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, seconds_max):
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (replicas: each rank runs the same workload)."""
+    return units_per_rank * world / seconds_max
+
+
 # ---------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------
@@ -556,13 +571,9 @@ def main():
         raise SystemExit("device status: a kernel timed out in the timed region")
     j = n_ev
 
-    elapsed_ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     sec_per_step = elapsed_ms / 1e3 / steps
-    value = wl.value(sec_per_step) * world
+    value = job_throughput(wl.value(sec_per_step), world, 1.0)
 
     kern_ms = {k: statistics.mean(e[ki][0].elapsed_time(e[ki][1]) for e in ev[:j])
                for ki, k in enumerate(wl.kernels)}
@@ -600,12 +611,9 @@ def main():
             wl.e2e_step(dev)
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b) / n_e2e
-        if dist is not None:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": wl.value(e_ms / 1e3) * world, "unit": wl.unit, "h2d_bytes_per_step": hb,
+        e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, dist, dev)
+        e2e = {"value": job_throughput(wl.value(e_ms / 1e3), world, 1.0), "unit": wl.unit,
+               "h2d_bytes_per_step": hb,
                "d2h_bytes_per_step": db, "ms_per_step": e_ms}
 
     cpu = None

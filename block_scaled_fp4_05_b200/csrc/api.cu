@@ -270,6 +270,15 @@ fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA
                                 fp4::noalloc_scratch_bytes(), FP4_GEMM_DECODE, stream);
 }
 
+fp4_status fp4_selftest_bounded_wait(fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_wait_selftest(reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fp4_status fp4_get_device_status(fp4_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

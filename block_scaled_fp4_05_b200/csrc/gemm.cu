@@ -68,7 +68,7 @@ constexpr int kThreads = 320;    // 10 warps: producer, MMA, 4 epilogue, 4 scale
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum : unsigned { ERR_FULL = 1u, ERR_EMPTY = 2u, ERR_ACC_FULL = 4u, ERR_ACC_EMPTY = 8u,
-                  ERR_DRAIN = 16u };
+                  ERR_DRAIN = 16u, ERR_SELFTEST = 32u };
 
 template <int BN, int STAGES>
 struct Cfg {
@@ -1179,6 +1179,21 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     }
 }
 
+// Self-test of the bounded wait used by every kernel above: one thread waits
+// on a barrier that nothing will ever complete.  The wait gives up after
+// kTimeoutNs, records the error word, and the kernel returns normally.
+__global__ void bounded_wait_selftest_kernel()
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        wait_bounded(smem_u32(&bar), 0, reinterpret_cast<volatile int*>(&abort_flag), ERR_SELFTEST);
+    }
+}
+
 // Sum of the stream-K partials of each output element in CTA order, times
 // alpha, to BF16.  Output D[m][n] (m < tokens, n < weight rows).
 template <int BN>
@@ -1451,6 +1466,12 @@ cudaError_t noalloc_scratch(void** out)
     if (dev < 64) cache[dev] = ptr;
     *out = ptr;
     return cudaSuccess;
+}
+
+cudaError_t launch_wait_selftest(cudaStream_t s)
+{
+    bounded_wait_selftest_kernel<<<1, 32, 0, s>>>();
+    return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_error_word(unsigned int* word)

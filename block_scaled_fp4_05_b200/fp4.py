@@ -71,6 +71,10 @@ def lib():
         L.fp4_gemm_workspace_bytes.argtypes = [c.c_int, i64, i64, i64]
         L.fp4_get_device_status.restype = c.c_int
         L.fp4_get_device_status.argtypes = [st]
+        L.fp4_selftest_bounded_wait.restype = c.c_int
+        L.fp4_selftest_bounded_wait.argtypes = [st]
+        L.fp4_gemm_decode_noalloc.restype = c.c_int
+        L.fp4_gemm_decode_noalloc.argtypes = [c.c_int, P, P, P, P, i64, i64, i64, P, P, i64, st]
         _lib = L
     return _lib
 
@@ -165,6 +169,10 @@ def fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace=None, kernel=GEMM_A
 
 def fp4_get_device_status(stream=None):
     return lib().fp4_get_device_status(_stream(stream))
+
+
+def fp4_selftest_bounded_wait(stream=None):
+    _check(lib().fp4_selftest_bounded_wait(_stream(stream)), "fp4_selftest_bounded_wait")
 
 
 # ---------------------------------------------------------------------------

@@ -225,6 +225,17 @@ fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA
  */
 fp4_status fp4_get_device_status(fp4_stream_t stream);
 
+/*
+ * Self-test of the failure path every kernel of this library uses: launches a
+ * one-thread kernel that waits on a barrier nothing will ever complete.  The
+ * bounded wait gives up after its time limit (2 s), records the timeout in
+ * the device error word and returns, without trapping, so the context stays
+ * usable.  After the stream reaches it, fp4_get_device_status reports
+ * FP4_ERR_TIMEOUT (and clears the word).  Not part of the method on the
+ * pages; a check of the library's fault handling.
+ */
+fp4_status fp4_selftest_bounded_wait(fp4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

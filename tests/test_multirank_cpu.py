@@ -1,0 +1,60 @@
+"""The N > 1 path of bench.py on CPU: two gloo ranks, each a replica with its
+own time; the job time is the slowest rank's and the throughput counts the
+units of every rank (weak scaling, no data-path collective)."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, results):
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [12.5, 20.0][rank]
+        worst = bench.max_over_ranks(local_ms, dist, "cpu")
+        units = 1000.0   # per-rank work per step
+        value = bench.job_throughput(units / (worst / 1e3), world, 1.0)
+        results[rank] = (worst, value)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_replica_aggregation():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    results = mgr.dict()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, results)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in range(world):
+        worst, value = results[r]
+        assert worst == 20.0
+        assert value == pytest.approx(2 * 1000.0 / 0.020)
+
+
+def test_single_rank_helpers():
+    import bench
+    assert bench.max_over_ranks(3.0) == 3.0
+    assert bench.job_throughput(10.0, 1, 2.0) == 5.0
