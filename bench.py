@@ -179,6 +179,12 @@ class SquareWorkload(Workload):
     """Quantize A and B (rowwise, along K) and D = A_hat B_hat^T, M=N=K=n."""
 
     def __init__(self, fmt, n, dev, sets=4, stream=None):
+        # quantize A and quantize B are independent: B runs on a second stream
+        # (a parallel branch in the captured graph) and the GEMM waits for both
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.stream2 = torch.cuda.Stream(device=dev)
+        self.fork = torch.cuda.Event()
+        self.join = torch.cuda.Event()
         self.fmt, self.n = fmt, n
         self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
         A, B = synth.square(n)
@@ -202,7 +208,7 @@ class SquareWorkload(Workload):
             else:
                 gA = gB = al = None
             groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Ad, pA, sA, gA, stream)])
-            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB, stream)])
+            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB, self.stream2)])
             groups.append([fp4.bind_gemm(fmt, pA, sA, pB, sB, n, n, n, al, D, None, fp4.GEMM_PREFILL,
                                          stream)])
             self.calls.append(groups)
@@ -222,6 +228,34 @@ class SquareWorkload(Workload):
 
     def value(self, sec_per_step):
         return self.flops / sec_per_step / 1e12
+
+    def step(self, i, ev=None):
+        calls = self.calls[i % len(self.calls)]
+        names = self.kernels
+        qa, qb = names.index("quantize_A"), names.index("quantize_B")
+        for k, group in enumerate(calls):
+            if k == qb:
+                continue
+            if k == qa:
+                # fork: B's quantization on the second stream, concurrently
+                self.fork.record(self.stream)
+                self.stream2.wait_event(self.fork)
+                with torch.cuda.stream(self.stream2):
+                    if ev is not None:
+                        ev[qb][0].record(self.stream2)
+                    for c in calls[qb]:
+                        c()
+                    if ev is not None:
+                        ev[qb][1].record(self.stream2)
+                self.join.record(self.stream2)
+            if ev is not None:
+                ev[k][0].record(self.stream)
+            for c in group:
+                c()
+            if ev is not None:
+                ev[k][1].record(self.stream)
+            if k == qa:
+                self.stream.wait_event(self.join)
 
     def e2e_setup(self, dev):
         A, B = self.host

@@ -313,6 +313,14 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32])
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+                 "r"(r[7])
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
@@ -763,18 +771,23 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 constexpr int PAIR_BN = 256;                 // N of the pair tile
 constexpr int PAIR_BHALF = PAIR_BN / 2;      // B rows staged by each CTA
 
-template <int STAGES>
+// Per stage, NVFP4 carries 4 scale chunks per 128 rows (one per K=64 MMA),
+// MXFP4 2 (one per two MMAs); the scale region of a stage is sized for its
+// format, so MXFP4 fits a sixth stage.
+template <int STAGES, bool MX>
 struct PairCfg {
+    static constexpr int NCH = MX ? 2 : 4;                          // scale chunks per 128 rows
     static constexpr int B_BYTES = PAIR_BHALF * BK_BYTES;           // 16 KB
-    static constexpr int SFB_BYTES = 2 * SFA_BYTES;                 // 256 B rows: 2 row tiles
-    static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int SFA_STAGE = NCH * SF_CHUNK;
+    static constexpr int SFB_STAGE = 2 * NCH * SF_CHUNK;            // 256 B rows: 2 row tiles
+    static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_STAGE + SFB_STAGE;
     static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
     static constexpr int OFF_B = A_BYTES;
     static constexpr int OFF_SFA = A_BYTES + B_BYTES;
-    static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + SFA_STAGE;
     static constexpr int SF_COL0 = PAIR_BN;                        // accumulator: columns [0, 256)
-    static constexpr int SFA_COLS = 16;
-    static constexpr int SF_COLS = SFA_COLS + 32;
+    static constexpr int SFA_COLS = 4 * NCH;
+    static constexpr int SF_COLS = SFA_COLS + 8 * NCH;
     static constexpr int TMEM_COLS = 512;
     static constexpr int NBARS = 5 * STAGES + 4;
     static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 512;
@@ -886,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const Params p)
 {
-    using C = PairCfg<STAGES>;
+    using C = PairCfg<STAGES, MX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -981,7 +994,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     if (nbh > 0)
                         bulk_load(st + C::OFF_SFB, sfb_row + ct0 * SF_CHUNK, sf_bytes, B_SFFULL(stage));
                     if (nbh > 1)
-                        bulk_load(st + C::OFF_SFB + SFA_BYTES, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
+                        bulk_load(st + C::OFF_SFB + C::SFA_STAGE, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
                                   sf_bytes, B_SFFULL(stage));
                     if (++stage == STAGES) {
                         stage = 0;
@@ -1127,9 +1140,9 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const int nch = MX ? nk / 2 : nk;
                 const uint32_t st = smem0 + stage * C::STAGE_BYTES + lane * 16;
                 const uint32_t tsf = tq + C::SF_COL0 + stage * C::SF_COLS;
-                uint32_t a[16];
+                uint32_t a[4 * C::NCH];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < C::NCH; ++j) {
                     uint4 v = make_uint4(0u, 0u, 0u, 0u);
                     if (j < nch && has_sfa) v = ld_shared_v4(st + C::OFF_SFA + j * SF_CHUNK);
                     a[4 * j] = v.x;
@@ -1137,21 +1150,26 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     a[4 * j + 2] = v.z;
                     a[4 * j + 3] = v.w;
                 }
-                tmem_st16(tsf, a);
-                uint32_t b[32];
+                uint32_t b[8 * C::NCH];
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < C::NCH; ++j)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         uint4 v = make_uint4(0u, 0u, 0u, 0u);
                         if (j < nch && h < nbh)
-                            v = ld_shared_v4(st + C::OFF_SFB + h * SFA_BYTES + j * SF_CHUNK);
+                            v = ld_shared_v4(st + C::OFF_SFB + h * C::SFA_STAGE + j * SF_CHUNK);
                         b[(j * 2 + h) * 4] = v.x;
                         b[(j * 2 + h) * 4 + 1] = v.y;
                         b[(j * 2 + h) * 4 + 2] = v.z;
                         b[(j * 2 + h) * 4 + 3] = v.w;
                     }
-                tmem_st32(tsf + C::SFA_COLS, b);
+                if constexpr (MX) {
+                    tmem_st8(tsf, a);
+                    tmem_st16(tsf + C::SFA_COLS, b);
+                } else {
+                    tmem_st16(tsf, a);
+                    tmem_st32(tsf + C::SFA_COLS, b);
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -1347,7 +1365,7 @@ template <int STAGES, bool MX>
 cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
                                int grid, cudaStream_t s)
 {
-    using C = PairCfg<STAGES>;
+    using C = PairCfg<STAGES, MX>;
     auto kern = fp4_gemm_pair_kernel<STAGES, MX>;
     static std::mutex mu;
     static uint64_t done_mask = 0;
@@ -1382,7 +1400,8 @@ cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, con
     return e;
 }
 
-constexpr int PAIR_STAGES = 5;
+constexpr int PAIR_STAGES_NV = 5;   // 38 KB per stage
+constexpr int PAIR_STAGES_MX = 6;   // 35 KB per stage
 
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
 {
@@ -1398,8 +1417,8 @@ cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaSt
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     const int64_t max_pairs = dev.sm_count / 2;
     const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
-    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES, true>(ta, tb, p, grid, s);
-    return launch_pair_kernel<PAIR_STAGES, false>(ta, tb, p, grid, s);
+    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true>(ta, tb, p, grid, s);
+    return launch_pair_kernel<PAIR_STAGES_NV, false>(ta, tb, p, grid, s);
 }
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
