@@ -39,8 +39,9 @@
 // Decode form (M <= 16 tokens): the operands are swapped so that the weight
 // rows fill the 128-row MMA side and the tokens form a 16-wide N side; the
 // (weight tile, K stage) work units are split evenly over the CTAs
-// (stream-K), each CTA writes FP32 partials per weight tile it touched, and a
-// reduction kernel sums them in a fixed order, applies alpha and writes BF16.
+// (stream-K), each CTA writes FP32 partials per weight tile it touched, and
+// the CTA that completes a tile sums its partials in a fixed (CTA) order,
+// applies alpha and writes BF16.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -106,6 +107,7 @@ struct Params {
     uint16_t* D;
     int64_t ldd;
     float* ws;
+    int* counters;             // stream-K: arrivals per (weight tile, lane quadrant)
 };
 
 // ------------------------------------------------------------------------
@@ -642,19 +644,56 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                                            packed[4 * i + 3]);
                 }
             } else {
+                static_assert(BN == 16, "the stream-K epilogue reads one 16-column chunk");
+                // FP32 partial of this segment; the CTA whose partial completes
+                // a weight tile (per 32-row lane quadrant) sums all partials of
+                // that tile in CTA order and writes the BF16 outputs.
                 float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
-#pragma unroll 1
-                for (int c = 0; c < BN / 16; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(trow + c * 16, r);
-                    tmem_wait_ld(r);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        slot[(c * 16 + j) * BM + row] = __uint_as_float(r[j]);
-                }
+                uint32_t r[16];
+                tmem_ld16(trow, r);
+                tmem_wait_ld(r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (j < p.rows_b) slot[j * BM + row] = __uint_as_float(r[j]);
+                __threadfence();
+                __syncwarp();
+                const int64_t G = gridDim.x;
+                const int64_t x0 = (int64_t)sg.tm * p.ks_total, x1 = x0 + p.ks_total - 1;
+                const int c0 = (int)(((x0 + 1) * G - 1) / p.units);
+                const int c1 = (int)(((x1 + 1) * G - 1) / p.units);
+                int* counter = p.counters + sg.tm * 4 + q;
+                int last = 0;
+                if (lane == 0) last = (atomicAdd(counter, 1) == c1 - c0) ? 1 : 0;
+                last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                if (last) {
+                    __threadfence();
+                    const int64_t n = (int64_t)sg.tm * BM + row;
+                    float sum[16];
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) sum[m] = 0.0f;
+                    for (int c = c0; c <= c1; ++c) {   // contributors in CTA order
+                        const int ubc = (int)(((int64_t)c * p.units) / G);
+                        const int slot_c = sg.tm - ubc / p.ks_total;
+                        const float* part = p.ws + ((int64_t)c * p.max_seg + slot_c) * (BN * BM) + row;
+                        float v[16];
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) v[m] = m < p.rows_b ? __ldcg(part + m * BM) : 0.0f;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) sum[m] = __fadd_rn(sum[m], v[m]);
+                    }
+                    if (n < p.rows_a) {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            if (m < p.rows_b) {
+                                const uint32_t b = pack_bf16x2(__fmul_rn(alpha, sum[m]), 0.0f);
+                                p.D[(int64_t)m * p.ldd + n] = (uint16_t)(b & 0xFFFFu);
+                            }
+                    }
+                    if (lane == 0) *counter = 0;   // ready for the next call
+                }
             }
             acc_phase ^= 1u;
         }
@@ -814,12 +853,6 @@ __device__ __forceinline__ void cluster_sync()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                      : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
-{
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-                 : "memory");
 }
 
 // Arrive on a barrier of the other CTA without a cluster-scope release
@@ -1212,34 +1245,6 @@ __global__ void bounded_wait_selftest_kernel()
     }
 }
 
-// Sum of the stream-K partials of each output element in CTA order, times
-// alpha, to BF16.  Output D[m][n] (m < tokens, n < weight rows).
-template <int BN>
-__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int max_seg, int units, int G,
-                                     int ks_total, int n_rows, int tokens,
-                                     const float* __restrict__ alpha_ptr, uint16_t* __restrict__ D,
-                                     int64_t ldd)
-{
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (int64_t)n_rows * tokens) return;
-    const int n = (int)(idx % n_rows);
-    const int m = (int)(idx / n_rows);
-    const int tm = n / BM, lane = n % BM;
-    const int64_t x0 = (int64_t)tm * ks_total, x1 = x0 + ks_total - 1;
-    const int c0 = (int)(((x0 + 1) * G - 1) / units);
-    const int c1 = (int)(((x1 + 1) * G - 1) / units);
-    float sum = 0.0f;
-    for (int c = c0; c <= c1; ++c) {
-        const int ubc = (int)(((int64_t)c * units) / G);
-        const int slot = tm - ubc / ks_total;
-        sum = __fadd_rn(sum, ws[(((int64_t)c * max_seg + slot) * BN + m) * BM + lane]);
-    }
-    const float a = alpha_ptr ? __ldg(alpha_ptr) : 1.0f;
-    const float v = __fmul_rn(a, sum);
-    uint32_t b = pack_bf16x2(v, 0.0f);
-    D[(int64_t)m * ldd + n] = (uint16_t)(b & 0xFFFFu);
-}
-
 // ------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------
@@ -1318,13 +1323,25 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
     return e;
 }
 
-constexpr int PREFILL_BN = 256, PREFILL_STAGES = 4;
 constexpr int DECODE_BN = 16, DECODE_STAGES = 8;
 
 int decode_max_seg(int units, int G, int ks_total)
 {
     const int span = (units + G - 1) / G;
     return (span - 1) / ks_total + 2;
+}
+
+// Workspace of the decode kernel: FP32 partials [CTA][segment][16][128],
+// then one arrival counter per (weight tile, lane quadrant).
+size_t decode_partials_bytes(int G, int max_seg)
+{
+    const size_t b = (size_t)G * max_seg * DECODE_BN * BM * sizeof(float);
+    return (b + 255) / 256 * 256;
+}
+
+size_t decode_counter_bytes(int64_t tiles)
+{
+    return ((size_t)tiles * 4 * sizeof(int) + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -1337,7 +1354,8 @@ size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count)
     const int ks_total = (int)((K + BK - 1) / BK);
     const int units = (int)((N + BM - 1) / BM) * ks_total;
     const int G = sm_count < units ? sm_count : units;
-    return (size_t)G * decode_max_seg(units, G, ks_total) * DECODE_BN * BM * sizeof(float);
+    return decode_partials_bytes(G, decode_max_seg(units, G, ks_total)) +
+           decode_counter_bytes((N + BM - 1) / BM);
 }
 
 static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t rows_b,
@@ -1357,6 +1375,7 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.D = a.D;
     p.ldd = a.ldd;
     p.ws = nullptr;
+    p.counters = nullptr;
     p.units = 0;
     p.max_seg = 0;
 }
@@ -1438,17 +1457,15 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     const int G = p.units < dev.sm_count ? p.units : dev.sm_count;
     p.max_seg = decode_max_seg(p.units, G, p.ks_total);
     p.ws = static_cast<float*>(a.ws);
-    cudaError_t e;
+    p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(a.ws) + decode_partials_bytes(G, p.max_seg));
+    cudaError_t e = cudaMemsetAsync(p.counters, 0, decode_counter_bytes(p.tiles_m), s);
+    if (e != cudaSuccess) {
+        set_last_error("cudaMemsetAsync(decode counters)", e);
+        return e;
+    }
     if (a.fmt == kMx)
-        e = launch_kernel<DECODE_BN, DECODE_STAGES, true, true>(tw, tx, p, G, s);
-    else
-        e = launch_kernel<DECODE_BN, DECODE_STAGES, false, true>(tw, tx, p, G, s);
-    if (e != cudaSuccess) return e;
-    const int64_t total = a.N * a.M;
-    const int threads = 256;
-    splitk_reduce_kernel<DECODE_BN><<<(unsigned)((total + threads - 1) / threads), threads, 0, s>>>(
-        p.ws, p.max_seg, p.units, G, p.ks_total, (int)a.N, (int)a.M, a.alpha, a.D, a.ldd);
-    return cudaGetLastError();
+        return launch_kernel<DECODE_BN, DECODE_STAGES, true, true>(tw, tx, p, G, s);
+    return launch_kernel<DECODE_BN, DECODE_STAGES, false, true>(tw, tx, p, G, s);
 }
 
 // ------------------------------------------------------------------------
