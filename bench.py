@@ -335,7 +335,7 @@ class DecodeWorkload(Workload):
         W = synth.decode_weight(N, K)
         A = synth.decode_activation(M, K)
         self.host = (A, W)
-        self.kernels = ["act_global_scale", "act_quantize", "gemm"]
+        self.kernels = ["act_quantize", "gemm"]
         self.calls, self.bufs = [], []
         Wd = _dev_bf16(W, dev)
         gW = fp4.global_scale(Wd)
@@ -348,9 +348,10 @@ class DecodeWorkload(Workload):
             D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = torch.empty((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
                              dtype=torch.uint8, device=dev)
+            # per call: S_global of the activation, its quantization and alpha in
+            # one launch, then the decode GEMM
             self.calls.append([
-                [fp4.bind_global_scale(Ad, gA, stream), fp4.bind_alpha(gA, gW, al, stream)],
-                [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA, stream)],
+                [fp4.bind_quantize_dynamic(Ad, pA, sA, gA, gW, al, stream)],
                 [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws, fp4.GEMM_DECODE, stream)],
             ])
             self.bufs.append((pW, sW, Ad, gA, al, pA, sA, D, ws))
@@ -359,11 +360,10 @@ class DecodeWorkload(Workload):
         wbytes = N * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, N, K)
         abytes = M * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, M, K)
         self.gemm_bytes = wbytes + abytes + M * N * 2
-        self.work = {"gemm": self.gemm_bytes, "act_quantize": M * K * 2 + abytes,
-                     "act_global_scale": M * K * 2}
-        self.bound = {"gemm": "hbm", "act_quantize": "hbm", "act_global_scale": "hbm"}
+        self.work = {"gemm": self.gemm_bytes, "act_quantize": 2 * M * K * 2 + abytes}
+        self.bound = {"gemm": "hbm", "act_quantize": "hbm"}
         self.flops = 2.0 * M * N * K
-        self.launches_per_step = 2 + 1 + 1 + 2   # amax+finalize, alpha, quantize, gemm+reduce
+        self.launches_per_step = 2   # dynamic activation quantizer, decode GEMM
         self.dominant = "gemm"
         self.l2_note = "rotating %d quantized weight copies (%.0f MB) > %d MB L2" % (
             sets, sets * wbytes / 1e6, L2_BYTES >> 20)

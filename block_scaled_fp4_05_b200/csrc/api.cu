@@ -152,6 +152,31 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
         fmt == FP4_NVFP4 ? global_scale : nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+fp4_status fp4_quantize_dynamic(fp4_format fmt, const void* in_bf16, int64_t rows, int64_t cols,
+                                int64_t ld, void* packed_out, void* scales_out, float* gs_out,
+                                const float* other_gs, float* alpha_out, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (fmt != FP4_NVFP4) return FP4_ERR_INVALID_ARG;
+    if (rows < 0 || cols < 0 || ld < cols || !gs_out) return FP4_ERR_INVALID_ARG;
+    if (alpha_out && !other_gs) return FP4_ERR_INVALID_ARG;
+    if (rows == 0 || cols == 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!in_bf16 || !packed_out || !scales_out) return FP4_ERR_INVALID_ARG;
+    if (cols % 64 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld % 8 != 0 || !aligned16(in_bf16) || !aligned16(packed_out) || !aligned16(scales_out))
+        return FP4_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(gs_out) & 3u) || (alpha_out && (reinterpret_cast<uintptr_t>(alpha_out) & 3u)) ||
+        (other_gs && (reinterpret_cast<uintptr_t>(other_gs) & 3u)))
+        return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_quantize_dynamic(
+        static_cast<const uint16_t*>(in_bf16), rows, cols, ld, static_cast<uint8_t*>(packed_out),
+        static_cast<uint8_t*>(scales_out), gs_out, other_gs, alpha_out,
+        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, float* alpha_out,
                                         fp4_stream_t stream)
 {

@@ -26,6 +26,9 @@ cudaError_t device_info(DeviceInfo* out);
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                         float* gs_out, cudaStream_t s);
 cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s);
+cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                    uint8_t* packed, uint8_t* scales, float* gs_out,
+                                    const float* other_gs, float* alpha_out, cudaStream_t s);
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
                             cudaStream_t s);

@@ -120,34 +120,24 @@ __device__ __forceinline__ uint32_t quantize8(uint4 v, float inv)
 // grid = (cols / 4k, ceil(rows / 128)).
 // ---------------------------------------------------------------------------
 template <int FMT>
-__global__ void __launch_bounds__(kThreads)
-quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
-                        const float* __restrict__ gs_ptr)
+__device__ __forceinline__ void rowwise_tile(const uint16_t* __restrict__ x, int64_t rows, int64_t cols,
+                                             int64_t ld, uint8_t* __restrict__ packed,
+                                             uint8_t* __restrict__ scales, int64_t rt, int64_t ct,
+                                             float gs, float denom, uint8_t* s_tile)
 {
     constexpr int KB = FMT == kMx ? 32 : 16;     // elements per block
-    constexpr int TILE_C = 4 * KB;               // columns per CTA
+    constexpr int TILE_C = 4 * KB;               // columns per tile
     constexpr int CPR = TILE_C / 8;              // 16-byte chunks per row
     constexpr int RPP = kThreads / CPR;          // rows per pass
     constexpr int PASSES = 128 / RPP;
     constexpr int CPB = KB / 8;                  // chunks per block
 
-    __shared__ __align__(16) uint8_t s_tile[512];
-
     const int tid = threadIdx.x;
     const int cc = tid % CPR;
     const int rsub = tid / CPR;
-    const int64_t ct = blockIdx.x;
-    const int64_t rt = blockIdx.y;
     const int64_t c0 = ct * TILE_C;
     const int64_t r0 = rt * 128;
     const int64_t nct = cols / TILE_C;
-
-    float gs = 1.0f, denom = 6.0f;
-    if (FMT == kNv) {
-        gs = __ldg(gs_ptr);
-        denom = __fmul_rn(6.0f, gs);
-    }
 
     uint4 v[PASSES];
 #pragma unroll
@@ -180,6 +170,152 @@ quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     if (tid < 32) {
         const uint4 t = reinterpret_cast<const uint4*>(s_tile)[tid];
         reinterpret_cast<uint4*>(scales + (rt * nct + ct) * 512)[tid] = t;
+    }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                        const float* __restrict__ gs_ptr)
+{
+    __shared__ __align__(16) uint8_t s_tile[512];
+    float gs = 1.0f, denom = 6.0f;
+    if (FMT == kNv) {
+        gs = __ldg(gs_ptr);
+        denom = __fmul_rn(6.0f, gs);
+    }
+    rowwise_tile<FMT>(x, rows, cols, ld, packed, scales, blockIdx.y, blockIdx.x, gs, denom, s_tile);
+}
+
+// ---------------------------------------------------------------------------
+// Dynamic NVFP4 quantization of a small tensor (decode activations) in one
+// launch: a cluster of CTAs reads the tensor once into registers, computes
+// its amax (each CTA's partial maximum stored into every CTA's shared memory
+// through DSMEM, one cluster barrier), S_global =
+// amax / 2688 (1 for an all-zero tensor) and optionally alpha = S_global *
+// other, then quantizes the register-resident values with that scale.
+// Thread t of the cluster owns the 16-byte chunks t, t + T, t + 2T, ... of the
+// row-major tensor (T = threads in the cluster), so every warp load and store
+// is contiguous; a lane pair holds one 16-element block and eight lanes one
+// 4-byte group of a scale tile.  Padding rows of the last 128-row scale tile
+// get zero scale bytes, written while the loads are in flight.  Tensors with
+// more chunks than the cluster holds in registers take the amax / quantize /
+// alpha kernels instead (launch_quantize_dynamic).
+// ---------------------------------------------------------------------------
+constexpr int kDynClusterMax = 16;   // non-portable size, used when the device can schedule it
+constexpr int kDynClusterMin = 8;
+constexpr int kDynThreads = 1024;
+constexpr int kDynRegChunks = 4;
+
+__global__ void __launch_bounds__(kDynThreads)
+quantize_dynamic_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
+                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
+                        float* __restrict__ gs_out, const float* __restrict__ other_gs,
+                        float* __restrict__ alpha_out)
+{
+    __shared__ uint32_t s_part[kDynClusterMax];
+    __shared__ uint32_t s_warp[kDynThreads / 32];
+    __shared__ float s_gs;
+
+    uint32_t rank, csize;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(csize));
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    // chunk indices fit 32 bits (at most kDynMaxChunks chunks)
+    const uint32_t T = csize * kDynThreads;
+    const uint32_t gt = rank * kDynThreads + tid;
+    const uint32_t cpr = (uint32_t)(cols / 8);     // 16-byte chunks per row = packed words per row
+    const uint32_t n = (uint32_t)rows * cpr;
+    const uint32_t G = cpr / 8;                    // scale groups per row
+    auto scale_word = [&](uint32_t r, uint32_t g) {
+        return reinterpret_cast<uint32_t*>(scales + ((size_t)(r / 128) * G + g) * 512 + (r % 32) * 16 +
+                                           ((r / 32) % 4) * 4);
+    };
+
+    // phase 1: load this thread's chunks, amax over the cluster
+    uint4 v[kDynRegChunks];
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < kDynRegChunks; ++j) {
+        const uint32_t u = j * T + gt;
+        v[j] = make_uint4(0u, 0u, 0u, 0u);
+        if (u < n) {
+            const uint32_t r = u / cpr;
+            v[j] = ld_stream(reinterpret_cast<const uint4*>(x + (int64_t)r * ld) + (u - r * cpr));
+        }
+    }
+    // zero scale bytes for the padding rows of the last 128-row tile:
+    // consecutive threads take consecutive words of a 512-byte scale tile
+    // (word k holds row (k % 4) * 32 + k / 4 of the tile)
+    {
+        const uint32_t rt = (uint32_t)(rows - 1) / 128, first_pad = (uint32_t)rows - rt * 128;
+        if (first_pad < 128) {
+            uint32_t* tile0 = reinterpret_cast<uint32_t*>(scales + (size_t)rt * G * 512);
+            for (uint32_t w = gt; w < G * 128; w += T) {
+                const uint32_t k = w % 128;
+                if ((k % 4) * 32 + k / 4 >= first_pad) tile0[w] = 0u;
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kDynRegChunks; ++j) m = max(m, absmax8(v[j]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) s_warp[tid >> 5] = m;
+    __syncthreads();
+    // every CTA's partial max goes to every CTA, so that after the barrier
+    // the maxima are read locally and no CTA touches another's shared
+    // memory again
+    if (tid < (int)csize) {
+        uint32_t b = 0;
+        for (int w = 0; w < kDynThreads / 32; ++w) b = max(b, s_warp[w]);
+        uint32_t dst;
+        asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(dst)
+                     : "r"((uint32_t)__cvta_generic_to_shared(&s_part[rank])), "r"(tid));
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(dst), "r"(b) : "memory");
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+    if (tid == 0) {
+        uint32_t b = 0;
+        for (uint32_t i = 0; i < csize; ++i) b = max(b, s_part[i]);
+        const float amax = __uint_as_float(b << 16);
+        const float gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+        s_gs = gs;
+        if (rank == 0) {
+            *gs_out = gs;
+            if (alpha_out) *alpha_out = __fmul_rn(gs, __ldg(other_gs));
+        }
+    }
+    __syncthreads();
+    const float gs = s_gs;
+    const float denom = __fmul_rn(6.0f, gs);
+
+    // phase 2: quantize the register-resident chunks
+    uint32_t* out32 = reinterpret_cast<uint32_t*>(packed);
+    const int gbase = lane & ~7;
+#pragma unroll
+    for (int j = 0; j < kDynRegChunks; ++j) {
+        const uint32_t u = j * T + gt;
+        if (j * T + (gt & ~31u) >= n) break;   // warp-uniform: no chunk of this warp left
+        uint32_t am = absmax8(v[j]);
+        am = max(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+        float inv;
+        const uint32_t sb = block_scale<kNv>(am, gs, denom, &inv);
+        const uint32_t q = quantize8(v[j], inv);
+        const uint32_t word = __shfl_sync(0xFFFFFFFFu, sb, gbase) |
+                              (__shfl_sync(0xFFFFFFFFu, sb, gbase + 2) << 8) |
+                              (__shfl_sync(0xFFFFFFFFu, sb, gbase + 4) << 16) |
+                              (__shfl_sync(0xFFFFFFFFu, sb, gbase + 6) << 24);
+        if (u < n) {
+            out32[u] = q;
+            if ((lane & 7) == 0) {
+                const uint32_t r = u / cpr;
+                *scale_word(r, (u - r * cpr) / 8) = word;
+            }
+        }
     }
 }
 
@@ -359,6 +495,70 @@ cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaS
 {
     alpha_kernel<<<1, 1, 0, s>>>(gsA, gsB, alpha);
     return cudaGetLastError();
+}
+
+namespace {
+
+// Cluster size for the dynamic quantizer: 16 CTAs when the device can place
+// such a cluster, else the portable 8.  Decided once per process.
+int dynamic_cluster_size()
+{
+    static int size = 0;
+    if (size) return size;
+    int chosen = kDynClusterMin;
+    if (cudaFuncSetAttribute(quantize_dynamic_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+        cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kDynClusterMax, 1, 1);
+        cfg.blockDim = dim3(kDynThreads, 1, 1);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kDynClusterMax;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, quantize_dynamic_kernel, &cfg) == cudaSuccess && n >= 1)
+            chosen = kDynClusterMax;
+    }
+    cudaGetLastError();
+    size = chosen;
+    return size;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                    uint8_t* packed, uint8_t* scales, float* gs_out,
+                                    const float* other_gs, float* alpha_out, cudaStream_t s)
+{
+    const int cl = dynamic_cluster_size();
+    if (rows * (cols / 8) > (int64_t)cl * kDynThreads * kDynRegChunks) {
+        // too large to stay in one cluster's registers: amax pass, then the
+        // rowwise quantizer and alpha as separate kernels
+        cudaError_t e = launch_amax(x, rows, cols, ld, gs_out, s);
+        if (e == cudaSuccess) e = launch_quantize(kNv, 0, x, rows, cols, ld, packed, scales, gs_out, s);
+        if (e == cudaSuccess && alpha_out) e = launch_alpha(gs_out, other_gs, alpha_out, s);
+        if (e != cudaSuccess) set_last_error("dynamic quantizer (multi-kernel) launch", e);
+        return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cl, 1, 1);
+    cfg.blockDim = dim3(kDynThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cl;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, quantize_dynamic_kernel, x, rows, cols, ld, packed, scales,
+                                       gs_out, other_gs, alpha_out);
+    if (e != cudaSuccess) set_last_error("dynamic quantizer launch", e);
+    return e;
 }
 
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,

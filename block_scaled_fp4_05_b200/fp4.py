@@ -60,6 +60,8 @@ def lib():
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
+        L.fp4_quantize_dynamic.restype = c.c_int
+        L.fp4_quantize_dynamic.argtypes = [c.c_int, P, i64, i64, i64, P, P, P, P, P, st]
         L.fp4_alpha_from_global_scales.restype = c.c_int
         L.fp4_alpha_from_global_scales.argtypes = [P, P, P, st]
         L.fp4_gemm.restype = c.c_int
@@ -144,6 +146,26 @@ def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream
                               _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
                               _dptr(global_scale, "global_scale"), _stream(stream)),
            "fp4_quantize")
+
+
+def fp4_quantize_dynamic(x, packed_out, scales_out, gs_out, other_gs=None, alpha_out=None,
+                         stream=None):
+    """NVFP4: S_global of x, rowwise quantization with it and optionally
+    alpha = S_global * other_gs, in one launch."""
+    assert x.dtype == torch.bfloat16
+    _check(lib().fp4_quantize_dynamic(NVFP4, _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                                      _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
+                                      _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"),
+                                      _dptr(alpha_out, "alpha_out"), _stream(stream)),
+           "fp4_quantize_dynamic")
+
+
+def bind_quantize_dynamic(x, packed_out, scales_out, gs_out, other_gs=None, alpha_out=None,
+                          stream=None):
+    return BoundCall("fp4_quantize_dynamic", NVFP4, _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                     _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
+                     _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"),
+                     _dptr(alpha_out, "alpha_out"), _stream(stream))
 
 
 def fp4_alpha_from_global_scales(gsA, gsB, alpha_out, stream=None):

@@ -146,6 +146,25 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
                         int64_t cols, int64_t ld, void* packed_out, void* scales_out,
                         const float* global_scale, fp4_stream_t stream);
 
+/*
+ * Dynamic NVFP4 quantization of a small tensor (e.g. the few rows of a decode
+ * activation) in a single launch: S_global of the tensor (as
+ * fp4_compute_global_scale), then the rowwise quantization with it (as
+ * fp4_quantize), and optionally alpha = S_global * (*other_gs) (as
+ * fp4_alpha_from_global_scales with the other operand's scale).  Results are
+ * identical to those three calls.  One cluster of 8 CTAs does the work, so it
+ * suits tensors of up to a few hundred thousand elements; larger tensors are
+ * correct but use only 8 SMs.
+ *   fmt      : FP4_NVFP4 only (MXFP4 needs no per-tensor scale: use
+ *              fp4_quantize); else FP4_ERR_INVALID_ARG
+ *   in_bf16  : device, rows x cols (ld), cols % 64 == 0, rows, cols > 0
+ *   gs_out   : device float, S_global written here
+ *   other_gs, alpha_out : device floats, both NULL or both set
+ */
+fp4_status fp4_quantize_dynamic(fp4_format fmt, const void* in_bf16, int64_t rows, int64_t cols,
+                                int64_t ld, void* packed_out, void* scales_out, float* gs_out,
+                                const float* other_gs, float* alpha_out, fp4_stream_t stream);
+
 /* alpha = gsA * gsB (FP32), the factor that restores both per-tensor scales
  * after the block-scaled product (NVFP4).  All three are device pointers. */
 fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, float* alpha_out,

@@ -169,3 +169,43 @@ def sampled_rows_check(orc, fmt, axis, x_bits, n_rows=48):
 def test_full_size_sweep_sampled(orc, fmt, axis, shape):
     x = synth.quant_sweep(*shape)
     sampled_rows_check(orc, fmt, axis, x)
+
+
+@pytest.mark.parametrize("shape", [(1, 8192), (4, 8192), (16, 8192), (16, 512), (3, 64), (1, 64),
+                                   (200, 1024), (33, 8192), (300, 1024)])
+def test_dynamic_quantize_matches_oracle(orc, shape):
+    # one call: S_global, quantization with it, alpha = S_global * other; small tensors
+    # take the single-launch cluster kernel, (33, 8192) and (300, 1024) the multi-kernel path
+    x = synth.normal_bf16(*shape, seed=28, outlier_factor=100.0)
+    rows, cols = shape
+    xd = to_dev_bf16(x)
+    packed = Guarded(rows * cols // 2)
+    scales = Guarded(fp4.fp4_scale_bytes(fp4.NVFP4, rows, cols), fill=0x5A)
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    other = to_dev_f32(0.0123)
+    alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_quantize_dynamic(xd, packed.view, scales.view, gs, other, alpha)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    assert packed.guards_intact() and scales.guards_intact()
+    g = orc.global_scale(x)
+    assert np.float32(gs.item()) == np.float32(g)
+    assert np.float32(alpha.item()) == np.float32(g) * np.float32(0.0123)
+    p_orc, s_orc = orc.quantize(fp4.NVFP4, fp4.ROWWISE, x, gs=g)
+    assert np.array_equal(packed.view.cpu().numpy().reshape(rows, cols // 2), p_orc)
+    assert np.array_equal(scales.view.cpu().numpy(), s_orc)
+
+
+def test_dynamic_quantize_all_zero_and_rejects_mx():
+    x = torch.zeros((4, 128), dtype=torch.bfloat16, device="cuda")
+    p = torch.empty((4, 64), dtype=torch.uint8, device="cuda")
+    s = torch.empty((fp4.fp4_scale_bytes(fp4.NVFP4, 4, 128),), dtype=torch.uint8, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_quantize_dynamic(x, p, s, gs)
+    torch.cuda.synchronize()
+    assert gs.item() == 1.0 and int(p.sum().item()) == 0
+    import ctypes
+    st = fp4.lib().fp4_quantize_dynamic(fp4.MXFP4, ctypes.c_void_p(x.data_ptr()), 4, 128, 128,
+                                        ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(s.data_ptr()),
+                                        ctypes.c_void_p(gs.data_ptr()), None, None, None)
+    assert st == 1
