@@ -346,7 +346,7 @@ class DecodeWorkload(Workload):
             al = torch.empty(1, dtype=torch.float32, device=dev)
             pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
             D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-            ws = torch.empty((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
+            ws = torch.zeros((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
                              dtype=torch.uint8, device=dev)
             # per call: S_global of the activation, its quantization and alpha in
             # one launch, then the decode GEMM

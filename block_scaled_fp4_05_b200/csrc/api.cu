@@ -74,7 +74,7 @@ constexpr int64_t kMaxRows = (int64_t)1 << 31;
 
 extern "C" {
 
-int fp4_abi_version(void) { return 1; }
+int fp4_abi_version(void) { return 2; }
 
 const char* fp4_last_error(void) { return fp4::g_last_error; }
 
@@ -88,6 +88,7 @@ const char* fp4_status_string(fp4_status s)
     case FP4_ERR_CUDA: return "FP4_ERR_CUDA";
     case FP4_ERR_TIMEOUT: return "FP4_ERR_TIMEOUT";
     case FP4_ERR_NO_DEVICE: return "FP4_ERR_NO_DEVICE";
+    case FP4_ERR_WORKSPACE: return "FP4_ERR_WORKSPACE";
     }
     return "FP4_ERR_UNKNOWN";
 }
@@ -233,12 +234,12 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
     const size_t need = fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
     bool decode = false;
     if (kernel == FP4_GEMM_DECODE) {
-        if (M > 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (M > 16 || need == 0) return FP4_ERR_UNSUPPORTED_SHAPE;   // need == 0: N beyond the counters
         if (!workspace || ws_bytes < need) return FP4_ERR_INVALID_ARG;
         if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
         decode = true;
     } else if (kernel == FP4_GEMM_AUTO) {
-        decode = M <= 16 && workspace && ws_bytes >= need && aligned16(workspace);
+        decode = M <= 16 && need > 0 && workspace && ws_bytes >= need && aligned16(workspace);
     }
     fp4::GemmArgs a;
     a.fmt = (int)fmt;
@@ -277,8 +278,15 @@ fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA
     if (M == 0 || N == 0 || K == 0)   // nothing that needs scratch
         return fp4_gemm_with_kernel(fmt, A, sA, B, sB, M, N, K, alpha, D, ldd, nullptr, 0,
                                     FP4_GEMM_PREFILL, stream);
-    const size_t need = fp4_gemm_workspace_bytes(fmt, M, N, K);
-    if (need == 0) return FP4_ERR_NO_DEVICE;
+    fp4::DeviceInfo dev;
+    const fp4_status dst = require_device(&dev);
+    if (dst != FP4_OK) return dst;
+    const size_t need = fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
+    if (need == 0) {
+        snprintf(fp4::g_last_error, sizeof fp4::g_last_error,
+                 "N = %lld is beyond the decode kernel's arrival counters (N <= 524288)", (long long)N);
+        return FP4_ERR_UNSUPPORTED_SHAPE;
+    }
     if (need > fp4::noalloc_scratch_bytes()) {
         snprintf(fp4::g_last_error, sizeof fp4::g_last_error,
                  "decode partials need %zu bytes, above the %zu-byte static scratch", need,
@@ -311,7 +319,11 @@ fp4_status fp4_get_device_status(fp4_stream_t stream)
     unsigned int word = 0;
     e = fp4::read_and_clear_error_word(&word);
     if (e != cudaSuccess) return from_cuda(e);
-    return word ? FP4_ERR_TIMEOUT : FP4_OK;
+    if (!word) return FP4_OK;
+    e = fp4::clear_noalloc_counters();
+    if (e != cudaSuccess) return from_cuda(e);
+    return (word & fp4::kErrorWorkspaceBit) && !(word & ~fp4::kErrorWorkspaceBit) ? FP4_ERR_WORKSPACE
+                                                                                     : FP4_ERR_TIMEOUT;
 }
 
 }  // extern "C"

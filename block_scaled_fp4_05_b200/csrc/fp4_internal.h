@@ -54,6 +54,12 @@ cudaError_t read_and_clear_error_word(unsigned int* word);
 cudaError_t launch_wait_selftest(cudaStream_t s);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** out);
+// Zeroes the decode counters of the static scratch (current device), after an
+// error left them in an unknown state.
+cudaError_t clear_noalloc_counters();
+// Bit of the device error word set by a decode call whose workspace counters
+// were out of range (not zeroed).
+constexpr unsigned int kErrorWorkspaceBit = 64u;
 int tensor_map_encoder_available();
 
 // Records the detail of a failure for fp4_last_error() (thread-local).

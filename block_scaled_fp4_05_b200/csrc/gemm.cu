@@ -37,11 +37,14 @@
 // (scale_vec::2X, E8M0) one chunk serves two, selected by scale-factor id 0/2.
 //
 // Decode form (M <= 16 tokens): the operands are swapped so that the weight
-// rows fill the 128-row MMA side and the tokens form a 16-wide N side; the
-// (weight tile, K stage) work units are split evenly over the CTAs
-// (stream-K), each CTA writes FP32 partials per weight tile it touched, and
+// rows fill the 128-row MMA side and the tokens form a 16-wide N side.  The
+// weight tiles are scheduled as stream-K followed by data-parallel tiles: the
+// (weight tile, K stage) units of the first sk_tiles tiles are split evenly
+// over the CTAs, each CTA writes FP32 partials per such tile it touched, and
 // the CTA that completes a tile sums its partials in a fixed (CTA) order,
-// applies alpha and writes BF16.
+// applies alpha and writes BF16; then every CTA runs whole tiles, written
+// straight from the accumulator.  The split-K reductions thus overlap the
+// whole-tile phase instead of trailing the kernel.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -69,7 +72,7 @@ constexpr int kThreads = 320;    // 10 warps: producer, MMA, 4 epilogue, 4 scale
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum : unsigned { ERR_FULL = 1u, ERR_EMPTY = 2u, ERR_ACC_FULL = 4u, ERR_ACC_EMPTY = 8u,
-                  ERR_DRAIN = 16u, ERR_SELFTEST = 32u };
+                  ERR_DRAIN = 16u, ERR_SELFTEST = 32u, ERR_WORKSPACE = kErrorWorkspaceBit };
 
 template <int BN, int STAGES>
 struct Cfg {
@@ -101,7 +104,8 @@ struct Params {
     int32_t sf_col_tiles;      // 512-byte scale tiles per 128-row group
     int32_t sfa_row_tiles, sfb_row_tiles;
     int32_t tiles_m, tiles_n;
-    int32_t units;             // stream-K: tiles_m * ks_total
+    int32_t units;             // stream-K: sk_tiles * ks_total
+    int32_t sk_tiles;          // stream-K: tiles split over the CTAs; the rest run whole
     int32_t max_seg;           // stream-K: partial slots per CTA
     const float* alpha;
     uint16_t* D;
@@ -214,6 +218,25 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+
+// Device-scope release-acquire atomic increment (returns the old value).
+__device__ __forceinline__ int atomic_add_acq_rel(int* p, int v)
+{
+    int old;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+// Programmatic dependent launch.  The GEMM kernels are launched so that they
+// may start while the kernel before them on the stream is still running;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible, and every thread that reads an operand, the scales or alpha, or
+// writes D or the workspace, passes it first.  Everything before it (barrier
+// set-up, tensor memory allocation, tensor-map prefetch) overlaps the
+// previous kernel.  Without the launch attribute it returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream (if launched with the attribute) begin.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -374,11 +397,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 struct Seg {
     int tm, tn, kb, ke, slot;
 };
+// In the decode schedule a segment that covers a whole tile has no other
+// contributor and is written straight to D.
 
 template <bool STREAM_K>
 struct Schedule {
     const Params& p;
-    int next_tile;   // prefill: next tile index
+    int next_tile;   // prefill: next tile index; decode: next whole tile
     int u, ue, ub;   // stream-K: unit cursor / range
     __device__ explicit Schedule(const Params& pp) : p(pp)
     {
@@ -387,6 +412,7 @@ struct Schedule {
             ub = (int)(((int64_t)blockIdx.x * p.units) / G);
             ue = (int)(((int64_t)(blockIdx.x + 1) * p.units) / G);
             u = ub;
+            next_tile = p.sk_tiles + blockIdx.x;
         } else {
             next_tile = blockIdx.x;
         }
@@ -394,14 +420,22 @@ struct Schedule {
     __device__ bool next(Seg& s)
     {
         if (STREAM_K) {
-            if (u >= ue) return false;
-            s.tm = u / p.ks_total;
             s.tn = 0;
-            s.kb = u % p.ks_total;
-            const int left = ue - u;
-            s.ke = min(p.ks_total, s.kb + left);
-            s.slot = s.tm - ub / p.ks_total;
-            u += s.ke - s.kb;
+            if (u < ue) {
+                s.tm = u / p.ks_total;
+                s.kb = u % p.ks_total;
+                const int left = ue - u;
+                s.ke = min(p.ks_total, s.kb + left);
+                s.slot = s.tm - ub / p.ks_total;
+                u += s.ke - s.kb;
+                return true;
+            }
+            if (next_tile >= p.tiles_m) return false;
+            s.tm = next_tile;
+            s.kb = 0;
+            s.ke = p.ks_total;
+            s.slot = 0;
+            next_tile += gridDim.x;
             return true;
         } else {
             if (next_tile >= p.tiles_m * p.tiles_n) return false;
@@ -476,6 +510,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
             const uint32_t bar0 = smem_u32(bars);
             const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
+            pdl_wait();
             Schedule<STREAM_K> sched(p);
             Seg sg;
             int stage = 0;
@@ -517,6 +552,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     }
                 }
             }
+            pdl_trigger();
             // Drain: the last min(issued, STAGES) stages may still be in flight
             // if the consumers stopped early; wait for their transactions.
             if (!ok || *abort_flag) {
@@ -600,7 +636,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         // ---------------- epilogue (warps 2..5) ----------------
         const int q = warp & 3;               // TMEM lane quadrant of this warp
         const int row = q * 32 + lane;        // accumulator row of this thread
-        const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+        pdl_wait();
+        const float alpha = p.alpha ? *p.alpha : 1.0f;
         const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
         Schedule<STREAM_K> sched(p);
         Seg sg;
@@ -645,20 +682,36 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             } else {
                 static_assert(BN == 16, "the stream-K epilogue reads one 16-column chunk");
-                // FP32 partial of this segment; the CTA whose partial completes
-                // a weight tile (per 32-row lane quadrant) sums all partials of
-                // that tile in CTA order and writes the BF16 outputs.
-                float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
                 uint32_t r[16];
                 tmem_ld16(trow, r);
                 tmem_wait_ld(r);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(acc_empty);
+                if (sg.kb == 0 && sg.ke == p.ks_total) {
+                    // whole tile: no other contributor
+                    const int64_t n = (int64_t)sg.tm * BM + row;
+                    if (n < p.rows_a) {
+#pragma unroll
+                        for (int m = 0; m < 16; ++m)
+                            if (m < p.rows_b) {
+                                const uint32_t b = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[m])), 0.0f);
+                                p.D[(int64_t)m * p.ldd + n] = (uint16_t)(b & 0xFFFFu);
+                            }
+                    }
+                    acc_phase ^= 1u;
+                    continue;
+                }
+                // FP32 partial of this segment; the CTA whose partial completes
+                // a weight tile (per 32-row lane quadrant) sums all partials of
+                // that tile in CTA order and writes the BF16 outputs.  Ordering:
+                // the lanes' partial stores, a warp barrier, then lane 0's
+                // release-acquire increment; the last arriver's lanes read the
+                // other partials after another warp barrier.
+                float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (j < p.rows_b) slot[j * BM + row] = __uint_as_float(r[j]);
-                __threadfence();
+                    if (j < p.rows_b) __stcg(slot + j * BM + row, __uint_as_float(r[j]));
                 __syncwarp();
                 const int64_t G = gridDim.x;
                 const int64_t x0 = (int64_t)sg.tm * p.ks_total, x1 = x0 + p.ks_total - 1;
@@ -666,23 +719,43 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 const int c1 = (int)(((x1 + 1) * G - 1) / p.units);
                 int* counter = p.counters + sg.tm * 4 + q;
                 int last = 0;
-                if (lane == 0) last = (atomicAdd(counter, 1) == c1 - c0) ? 1 : 0;
+                if (lane == 0) {
+                    const int old = atomic_add_acq_rel(counter, 1);
+                    last = old == c1 - c0 ? 1 : 0;
+                    if (old < 0 || old > c1 - c0) atomicOr(&g_fp4_error_word, ERR_WORKSPACE);
+                }
                 last = __shfl_sync(0xFFFFFFFFu, last, 0);
                 if (last) {
-                    __threadfence();
+                    __syncwarp();
                     const int64_t n = (int64_t)sg.tm * BM + row;
                     float sum[16];
 #pragma unroll
                     for (int m = 0; m < 16; ++m) sum[m] = 0.0f;
-                    for (int c = c0; c <= c1; ++c) {   // contributors in CTA order
-                        const int ubc = (int)(((int64_t)c * p.units) / G);
-                        const int slot_c = sg.tm - ubc / p.ks_total;
-                        const float* part = p.ws + ((int64_t)c * p.max_seg + slot_c) * (BN * BM) + row;
-                        float v[16];
+                    // contributors in CTA order, up to four partial rows in
+                    // flight at a time; this CTA's own values come from registers
+                    for (int cb = c0; cb <= c1; cb += 4) {
+                        float v[4][16];
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) v[m] = m < p.rows_b ? __ldcg(part + m * BM) : 0.0f;
+                        for (int i = 0; i < 4; ++i) {
+                            const int c = cb + i;
+                            if (c > c1) break;
+                            if (c == (int)blockIdx.x) {
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) sum[m] = __fadd_rn(sum[m], v[m]);
+                                for (int m = 0; m < 16; ++m) v[i][m] = __uint_as_float(r[m]);
+                                continue;
+                            }
+                            const int ubc = (int)(((int64_t)c * p.units) / G);
+                            const int slot_c = sg.tm - ubc / p.ks_total;
+                            const float* part = p.ws + ((int64_t)c * p.max_seg + slot_c) * (BN * BM) + row;
+#pragma unroll
+                            for (int m = 0; m < 16; ++m) v[i][m] = m < p.rows_b ? __ldcg(part + m * BM) : 0.0f;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            if (cb + i > c1) break;
+#pragma unroll
+                            for (int m = 0; m < 16; ++m) sum[m] = __fadd_rn(sum[m], v[i][m]);
+                        }
                     }
                     if (n < p.rows_a) {
 #pragma unroll
@@ -995,6 +1068,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            pdl_wait();
             for (int t = pair; ok && t < tiles; t += npairs) {
                 const int tm = t % p.tiles_m, tn = t / p.tiles_m;
                 const int rta = tm * 2 + (int)rank;                // this CTA's 128-row A tile
@@ -1035,6 +1109,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                 }
             }
+            pdl_trigger();
             // On a give-up, give loads already issued time to land before the
             // CTAs meet at the final cluster barrier.
             if (!ok || *abort_flag) spin_ns(200000);
@@ -1103,7 +1178,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         // ---------------- epilogue (warps 2..5, both CTAs) ----------------
         const int q = warp & 3;
         const int row = q * 32 + lane;
-        const float alpha = p.alpha ? __ldg(p.alpha) : 1.0f;
+        pdl_wait();
+        const float alpha = p.alpha ? *p.alpha : 1.0f;
         const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
         const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
@@ -1305,8 +1381,17 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
         set_last_error("cudaFuncSetAttribute(max dynamic shared memory)", e);
         return e;
     }
-    fp4_gemm_kernel<BN, STAGES, MX, STREAM_K><<<grid, kThreads, C::SMEM, s>>>(ta, tb, p);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>, ta, tb, p);
     if (e != cudaSuccess) {
         cudaFuncAttributes fa{};
         cudaFuncGetAttributes(&fa, fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>);
@@ -1323,25 +1408,53 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
     return e;
 }
 
-constexpr int DECODE_BN = 16, DECODE_STAGES = 8;
+constexpr int DECODE_BN = 16, DECODE_STAGES = 8;    // 22 KB per stage
 
 int decode_max_seg(int units, int G, int ks_total)
 {
+    if (units == 0) return 1;
     const int span = (units + G - 1) / G;
     return (span - 1) / ks_total + 2;
 }
 
-// Workspace of the decode kernel: FP32 partials [CTA][segment][16][128],
-// then one arrival counter per (weight tile, lane quadrant).
+// Decode schedule: G CTAs; the first sk_tiles weight tiles are split over all
+// CTAs by K stage (stream-K), the remaining tiles (a multiple of G) run whole.
+// sk_tiles is the remainder of tiles / G, plus G more when that remainder
+// would give the CTAs fewer than two K stages each, so that no tile has a
+// crowd of one-stage contributors.  Fewer tiles than CTAs: all stream-K.
+struct DecodeSchedule {
+    int G, sk_tiles, max_seg;
+};
+
+DecodeSchedule decode_schedule(int64_t tiles, int ks_total, int sm_count)
+{
+    DecodeSchedule d;
+    const int64_t units = tiles * ks_total;
+    d.G = (int)(units < sm_count ? units : sm_count);
+    if (tiles <= d.G) {
+        d.sk_tiles = (int)tiles;
+    } else {
+        int64_t sk = tiles % d.G;
+        if (sk > 0 && sk * ks_total < 2 * (int64_t)d.G) sk += d.G;
+        d.sk_tiles = (int)sk;
+    }
+    d.max_seg = decode_max_seg(d.sk_tiles * ks_total, d.G, ks_total);
+    return d;
+}
+
+// Workspace of the decode kernel: a fixed 64 KB block of arrival counters,
+// one per (weight tile, lane quadrant), at offset 0 for every shape, then the
+// FP32 partials [CTA][segment][16][128].  The counters must be zero when a
+// call starts and every completed call leaves them zero, so a workspace that
+// was zeroed once serves any sequence of shapes: the partials of one shape
+// never overlap the counters of another.
+constexpr size_t kDecodeCounterBytes = 65536;
+constexpr int64_t kDecodeMaxTiles = kDecodeCounterBytes / (4 * sizeof(int));   // N <= 524288
+
 size_t decode_partials_bytes(int G, int max_seg)
 {
     const size_t b = (size_t)G * max_seg * DECODE_BN * BM * sizeof(float);
     return (b + 255) / 256 * 256;
-}
-
-size_t decode_counter_bytes(int64_t tiles)
-{
-    return ((size_t)tiles * 4 * sizeof(int) + 255) / 256 * 256;
 }
 
 }  // namespace
@@ -1351,11 +1464,10 @@ int tensor_map_encoder_available() { return encoder() != nullptr; }
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count)
 {
     if (M > DECODE_BN || M <= 0 || N <= 0 || K <= 0 || sm_count <= 0) return 0;
+    if ((N + BM - 1) / BM > kDecodeMaxTiles) return 0;
     const int ks_total = (int)((K + BK - 1) / BK);
-    const int units = (int)((N + BM - 1) / BM) * ks_total;
-    const int G = sm_count < units ? sm_count : units;
-    return decode_partials_bytes(G, decode_max_seg(units, G, ks_total)) +
-           decode_counter_bytes((N + BM - 1) / BM);
+    const DecodeSchedule d = decode_schedule((N + BM - 1) / BM, ks_total, sm_count);
+    return kDecodeCounterBytes + decode_partials_bytes(d.G, d.max_seg);
 }
 
 static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t rows_b,
@@ -1377,6 +1489,7 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.ws = nullptr;
     p.counters = nullptr;
     p.units = 0;
+    p.sk_tiles = 0;
     p.max_seg = 0;
 }
 
@@ -1407,13 +1520,15 @@ cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, con
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
     if (e != cudaSuccess) set_last_error("pair GEMM kernel launch", e);
     return e;
@@ -1453,28 +1568,27 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     fill_common(p, a, a.N, a.M, a.sB, a.sA);
     p.tiles_m = (int32_t)((a.N + BM - 1) / BM);
     p.tiles_n = 1;
-    p.units = p.tiles_m * p.ks_total;
-    const int G = p.units < dev.sm_count ? p.units : dev.sm_count;
-    p.max_seg = decode_max_seg(p.units, G, p.ks_total);
-    p.ws = static_cast<float*>(a.ws);
-    p.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(a.ws) + decode_partials_bytes(G, p.max_seg));
-    cudaError_t e = cudaMemsetAsync(p.counters, 0, decode_counter_bytes(p.tiles_m), s);
-    if (e != cudaSuccess) {
-        set_last_error("cudaMemsetAsync(decode counters)", e);
-        return e;
-    }
+    const DecodeSchedule d = decode_schedule(p.tiles_m, p.ks_total, dev.sm_count);
+    const int G = d.G;
+    p.sk_tiles = d.sk_tiles;
+    p.units = d.sk_tiles * p.ks_total;
+    p.max_seg = d.max_seg;
+    // the counters start at zero (caller's contract) and the kernel leaves
+    // them at zero
+    p.counters = static_cast<int*>(a.ws);
+    p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + kDecodeCounterBytes);
     if (a.fmt == kMx)
         return launch_kernel<DECODE_BN, DECODE_STAGES, true, true>(tw, tx, p, G, s);
     return launch_kernel<DECODE_BN, DECODE_STAGES, false, true>(tw, tx, p, G, s);
 }
 
 // ------------------------------------------------------------------------
-// Allocation-free decode: the split-K partials go to a fixed, file-scope
-// device array instead of a caller-provided workspace.  Every device that
-// loads the library holds these bytes until the process exits.  Successive
-// calls share the array and it keeps the last call's partials; nothing in it
-// needs to start at zero (each CTA writes every partial it later reads), but
-// two such calls that overlap on the GPU (different streams) race on it.
+// Allocation-free decode: the counters and split-K partials go to a fixed,
+// file-scope device array instead of a caller-provided workspace.  Every
+// device that loads the library holds these bytes until the process exits.
+// The array is zero at load, which is the state the counters need, and each
+// completed call leaves them zero; two such calls that overlap on the GPU
+// (different streams) race on it.
 // ------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
@@ -1502,6 +1616,16 @@ cudaError_t noalloc_scratch(void** out)
     if (dev < 64) cache[dev] = ptr;
     *out = ptr;
     return cudaSuccess;
+}
+
+cudaError_t clear_noalloc_counters()
+{
+    void* ptr = nullptr;
+    cudaError_t e = noalloc_scratch(&ptr);
+    if (e != cudaSuccess) return e;
+    e = cudaMemset(ptr, 0, kDecodeCounterBytes);
+    if (e != cudaSuccess) return e;
+    return cudaDeviceSynchronize();
 }
 
 cudaError_t launch_wait_selftest(cudaStream_t s)

@@ -27,6 +27,11 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// Lets a kernel launched after this one with programmatic stream
+// serialization (the GEMMs) start its set-up; it still waits for this
+// kernel's completion before reading anything this kernel writes.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint4 ld_stream(const uint4* p)
 {
     uint4 v;
@@ -180,6 +185,7 @@ quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
                         const float* __restrict__ gs_ptr)
 {
     __shared__ __align__(16) uint8_t s_tile[512];
+    pdl_trigger();
     float gs = 1.0f, denom = 6.0f;
     if (FMT == kNv) {
         gs = __ldg(gs_ptr);
@@ -205,7 +211,7 @@ quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
 // ---------------------------------------------------------------------------
 constexpr int kDynClusterMax = 16;   // non-portable size, used when the device can schedule it
 constexpr int kDynClusterMin = 8;
-constexpr int kDynThreads = 1024;
+constexpr int kDynThreads = 512;    // leaves room on the SM for a GEMM CTA launched early
 constexpr int kDynRegChunks = 4;
 
 __global__ void __launch_bounds__(kDynThreads)
@@ -218,6 +224,7 @@ quantize_dynamic_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     __shared__ uint32_t s_warp[kDynThreads / 32];
     __shared__ float s_gs;
 
+    pdl_trigger();
     uint32_t rank, csize;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
     asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(csize));
@@ -341,6 +348,7 @@ quantize_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     __shared__ __align__(16) uint16_t s_in[TILE_K][128];
     __shared__ __align__(16) uint8_t s_out[128][OUT_BYTES];
     __shared__ __align__(16) uint8_t s_tile[512];
+    pdl_trigger();
 
     const int tid = threadIdx.x;
     const int64_t kt = blockIdx.x;        // scale-column tile (blocked direction)

@@ -19,6 +19,7 @@ FP4_OK = 0
 STATUS_NAMES = {
     0: "FP4_OK", 1: "FP4_ERR_INVALID_ARG", 2: "FP4_ERR_UNSUPPORTED_SHAPE",
     3: "FP4_ERR_MISALIGNED", 4: "FP4_ERR_CUDA", 5: "FP4_ERR_TIMEOUT", 6: "FP4_ERR_NO_DEVICE",
+    7: "FP4_ERR_WORKSPACE",
 }
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -224,7 +225,7 @@ def gemm(fmt, A, sA, B, sB, K, alpha=None, kernel=GEMM_AUTO, out=None, workspace
     if workspace is None and kernel != GEMM_PREFILL:
         nb = fp4_gemm_workspace_bytes(fmt, M, N, K)
         if nb:
-            workspace = torch.empty((nb,), dtype=torch.uint8, device=A.device)
+            workspace = torch.zeros((nb,), dtype=torch.uint8, device=A.device)
     fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace, kernel, stream)
     return D
 

@@ -75,7 +75,8 @@ typedef enum {
     FP4_ERR_MISALIGNED = 3,        /* pointer or leading dimension not 16-byte aligned */
     FP4_ERR_CUDA = 4,              /* a CUDA runtime call or launch failed */
     FP4_ERR_TIMEOUT = 5,           /* a kernel gave up on a bounded wait (see fp4_get_device_status) */
-    FP4_ERR_NO_DEVICE = 6          /* no usable sm_100 device */
+    FP4_ERR_NO_DEVICE = 6,         /* no usable sm_100 device */
+    FP4_ERR_WORKSPACE = 7          /* the decode workspace's counters were not zero (see fp4_gemm) */
 } fp4_status;
 
 typedef enum {
@@ -84,7 +85,7 @@ typedef enum {
     FP4_GEMM_DECODE = 2   /* swap-AB, stream-K kernel for M <= 16 plus a split-K reduction */
 } fp4_gemm_kernel;
 
-/* Version of this ABI (incremented on any signature change). */
+/* Version of this ABI (incremented on any signature or contract change). */
 int fp4_abi_version(void);
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -183,10 +184,22 @@ fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, floa
  *   D : BF16 [M x N], leading dimension ldd (elements, ldd >= N, ldd % 8 == 0)
  *   workspace / ws_bytes : scratch for the decode kernel's split-K partials
  *          (fp4_gemm_workspace_bytes); may be NULL / 0, then the prefill
- *          kernel runs for every M.
+ *          kernel runs for every M.  Its first 64 KB hold arrival counters
+ *          that must be zero when a call starts: zero the whole workspace
+ *          once after allocating it (cudaMemset); every call that completes
+ *          leaves the counters zero again, for any later shape.  A call that
+ *          finds a counter out of range records it and fp4_get_device_status
+ *          returns FP4_ERR_WORKSPACE; after that, or after FP4_ERR_TIMEOUT,
+ *          zero the workspace again.  Two calls that run at the same time
+ *          need two workspaces.
  * Requires K % 64 == 0 (NVFP4) or K % 128 == 0 (MXFP4) and N % 8 == 0.  M and
  * N tails are handled inside the kernels.  M == 0 or N == 0 is a no-op;
  * K == 0 writes zeros.
+ *
+ * The kernels are launched with programmatic stream serialization: one may
+ * start its set-up while the previous kernel on the stream is still running,
+ * and reads no operand, scale or alpha and writes no output before that
+ * kernel has completed, so stream order is kept.
  */
 fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B,
                     const void* sB, int64_t M, int64_t N, int64_t K, const float* alpha,
@@ -194,15 +207,16 @@ fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B
                     fp4_stream_t stream);
 
 /* Same as fp4_gemm with an explicit kernel choice.  FP4_GEMM_DECODE needs
- * M <= 16 and a workspace of fp4_gemm_workspace_bytes bytes (else
- * FP4_ERR_INVALID_ARG / FP4_ERR_UNSUPPORTED_SHAPE). */
+ * M <= 16, N <= 524288 and a workspace of fp4_gemm_workspace_bytes bytes
+ * (else FP4_ERR_UNSUPPORTED_SHAPE / FP4_ERR_INVALID_ARG). */
 fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, const void* B,
                                 const void* sB, int64_t M, int64_t N, int64_t K,
                                 const float* alpha, void* D, int64_t ldd, void* workspace,
                                 size_t ws_bytes, fp4_gemm_kernel kernel, fp4_stream_t stream);
 
 /* Workspace bytes the decode kernel needs for this shape on the current
- * device (0 when the decode kernel does not apply, i.e. M > 16). */
+ * device: 64 KB of counters plus the split-K partials (0 when the decode
+ * kernel does not apply, i.e. M > 16 or N > 524288). */
 size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K);
 
 /*
@@ -223,9 +237,11 @@ size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K)
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
- *  - All calls share the array and it keeps the last call's contents (nothing
- *    in it has to start at zero).  Calls that overlap on the GPU (e.g. on two
- *    streams at once) race on it: serialize them.
+ *  - All calls share the array.  It is zero when the library loads, and its
+ *    counters (see fp4_gemm's workspace) are zero again after every call
+ *    that completes; fp4_get_device_status zeroes them after reporting an
+ *    error.  Calls that overlap on the GPU (e.g. on two streams at once) race
+ *    on it: serialize them.
  *  - Shapes whose partials exceed 4 MiB (fp4_gemm_workspace_bytes) are
  *    rejected with FP4_ERR_UNSUPPORTED_SHAPE and an fp4_last_error() message;
  *    M > 16 is rejected the same way.  (N = 28672, K = 8192 needs 3.6 MB on
@@ -239,8 +255,11 @@ fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA
 /*
  * Synchronizes `stream`, then reports and clears the device error word of the
  * current device: FP4_ERR_TIMEOUT if a kernel of this library gave up on a
- * bounded wait since the last call (its outputs are then unspecified), else
- * FP4_OK; FP4_ERR_CUDA if the synchronization itself failed.
+ * bounded wait since the last call (its outputs are then unspecified),
+ * FP4_ERR_WORKSPACE if a decode call found its workspace counters not zero
+ * (outputs unspecified), else FP4_OK; FP4_ERR_CUDA if the synchronization
+ * itself failed.  After an error it also zeroes the counters of the static
+ * scratch of fp4_gemm_decode_noalloc.
  */
 fp4_status fp4_get_device_status(fp4_stream_t stream);
 

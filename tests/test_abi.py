@@ -13,7 +13,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.fp4_abi_version() == 1
+    assert L.fp4_abi_version() == 2
 
 
 def test_status_strings():

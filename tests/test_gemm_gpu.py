@@ -76,7 +76,10 @@ def test_prefill_ragged_shapes(orc, fmt, MNK):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("MNK", [(1, 256, 512), (4, 1000, 1024), (16, 1024, 8192), (7, 136, 384)])
+# (16, 38400, 1024) and (9, 38400, 1088): more weight tiles than SMs, so the
+# decode schedule runs stream-K tiles and then whole tiles; 1088 adds a K tail
+@pytest.mark.parametrize("MNK", [(1, 256, 512), (4, 1000, 1024), (16, 1024, 8192), (7, 136, 384),
+                                 (16, 38400, 1024), (9, 38400, 1088)])
 def test_decode_kernel_shapes(orc, fmt, MNK):
     M, N, K = MNK
     if K % (64 if fmt == fp4.NVFP4 else 128):
@@ -89,6 +92,46 @@ def test_decode_kernel_shapes(orc, fmt, MNK):
     assert_gemm_close(D, D_orc, S, "decode %s" % (MNK,))
     D2 = run_gpu_gemm(fmt, pA, sA, pW, sW, K, alpha, fp4.GEMM_PREFILL)
     assert_gemm_close(D2, D_orc, S, "prefill-on-decode-shape %s" % (MNK,))
+
+
+def test_decode_workspace_reused_across_shapes_stays_zeroed(orc):
+    # one workspace, zeroed once, serves a sequence of shapes: every call
+    # leaves the arrival counters (first 64 KB) at zero again
+    fmt = fp4.NVFP4
+    shapes = [(16, 1024, 8192), (3, 28672 // 4, 2048), (16, 1024, 8192), (1, 136, 384)]
+    nb = max(fp4.fp4_gemm_workspace_bytes(fmt, *s) for s in shapes)
+    ws = torch.zeros((nb,), dtype=torch.uint8, device="cuda")
+    for i, (M, N, K) in enumerate(shapes):
+        A = synth.normal_bf16(M, K, seed=40 + i, outlier_factor=100.0)
+        W = synth.normal_bf16(N, K, seed=40 + i, tensor_id=1, sigma=0.02)
+        pA, sA, pW, sW, alpha = oracle_operands(orc, fmt, A, W)
+        D = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        fp4.fp4_gemm(fmt, to_dev_u8(pA), to_dev_u8(sA), to_dev_u8(pW), to_dev_u8(sW), M, N, K,
+                     to_dev_f32(alpha), D, ws, kernel=fp4.GEMM_DECODE)
+        torch.cuda.synchronize()
+        assert fp4.fp4_get_device_status() == 0
+        assert int(ws[:65536].count_nonzero().item()) == 0
+        if N * K <= 1024 * 8192:
+            D_orc, S = orc.gemm(fmt, pA, sA, pW, sW, alpha=alpha)
+            assert_gemm_close(bf16_dev_to_f64(D), D_orc, S, "decode reuse %s" % ((M, N, K),))
+
+
+def test_decode_workspace_not_zeroed_is_reported():
+    # counters holding garbage: the kernel records it (no wait depends on
+    # them) and the status call reports FP4_ERR_WORKSPACE
+    fmt, M, N, K = fp4.NVFP4, 4, 512, 1024
+    A = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device="cuda")
+    W = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device="cuda")
+    sA = torch.full((fp4.fp4_scale_bytes(fmt, M, K),), 0x38, dtype=torch.uint8, device="cuda")
+    sW = torch.full((fp4.fp4_scale_bytes(fmt, N, K),), 0x38, dtype=torch.uint8, device="cuda")
+    ws = torch.full((fp4.fp4_gemm_workspace_bytes(fmt, M, N, K),), 0x7B, dtype=torch.uint8, device="cuda")
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fp4.fp4_gemm(fmt, A, sA, W, sW, M, N, K, None, D, ws, kernel=fp4.GEMM_DECODE)
+    assert fp4.fp4_get_device_status() == 7
+    assert fp4.fp4_get_device_status() == 0   # cleared
+    ws.zero_()
+    fp4.fp4_gemm(fmt, A, sA, W, sW, M, N, K, None, D, ws, kernel=fp4.GEMM_DECODE)
+    assert fp4.fp4_get_device_status() == 0
 
 
 def test_k_zero_and_empty():
