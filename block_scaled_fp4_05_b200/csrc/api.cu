@@ -207,8 +207,11 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
 {
     fp4::g_last_error[0] = 0;
     if (!valid_fmt(fmt)) return FP4_ERR_INVALID_ARG;
+    const int flags = (int)kernel & ~0xFF;
+    kernel = (fp4_gemm_kernel)((int)kernel & 0xFF);
     if (kernel != FP4_GEMM_AUTO && kernel != FP4_GEMM_PREFILL && kernel != FP4_GEMM_DECODE)
         return FP4_ERR_INVALID_ARG;
+    if (flags & ~(int)FP4_GEMM_B_STATIC) return FP4_ERR_INVALID_ARG;
     if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
     if (M == 0 || N == 0) return FP4_OK;
     if (!D) return FP4_ERR_INVALID_ARG;
@@ -255,6 +258,7 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
     a.ldd = ldd;
     a.ws = workspace;
     a.ws_bytes = ws_bytes;
+    a.b_static = (flags & FP4_GEMM_B_STATIC) != 0;
     const cudaError_t e = decode ? fp4::launch_gemm_decode(a, dev, s) : fp4::launch_gemm_prefill(a, dev, s);
     return from_cuda(e);
 }

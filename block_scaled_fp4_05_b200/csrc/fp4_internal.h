@@ -46,6 +46,7 @@ struct GemmArgs {
     int64_t ldd;
     void* ws;
     size_t ws_bytes;
+    bool b_static;      // B and sB not written by a kernel still running on the stream
 };
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);

@@ -106,6 +106,7 @@ struct Params {
     int32_t tiles_m, tiles_n;
     int32_t units;             // stream-K: sk_tiles * ks_total
     int32_t sk_tiles;          // stream-K: tiles split over the CTAs; the rest run whole
+    int32_t a_static;          // A side not written by the previous kernel: prefetch it
     int32_t max_seg;           // stream-K: partial slots per CTA
     const float* alpha;
     uint16_t* D;
@@ -510,6 +511,52 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
             const uint32_t bar0 = smem_u32(bars);
             const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
+            // scale row tiles of B that exist for a tile
+            auto count_nbh = [&](const Seg& g) {
+                const int rtb0 = (g.tn * BN) / 128;
+                int nbh = 0;
+                for (int h = 0; h < C::BH; ++h)
+                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
+                return nbh;
+            };
+            // Requests the A side (A tile + its scales) and/or the B side of
+            // K stage ks of segment g into ring slot stg; `expect` posts the
+            // stage's full byte count on its barrier.
+            auto issue = [&](int stg, const Seg& g, int ks, int nbh, bool a_side, bool b_side, bool expect) {
+                const uint32_t fb = bar0 + 8u * stg;
+                const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                const int nch = MX ? nk / 2 : nk;
+                const int ct0 = MX ? ks * 2 : ks * 4;   // first 512-byte scale chunk of the stage
+                const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
+                const uint32_t st = smem0 + stg * C::STAGE_BYTES;
+                if (expect) mbar_arrive_expect_tx(fb, A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
+                if (a_side) {
+                    tma_load_2d(&tmA, fb, st, ks * BK_BYTES, g.tm * BM);
+                    bulk_load(st + C::OFF_SFA, p.sfa + g.tm * sf_row_bytes + ct0 * SF_CHUNK, sf_bytes, fb);
+                }
+                if (b_side) {
+                    const uint8_t* sfb_row = p.sfb + ((g.tn * BN) / 128) * sf_row_bytes;
+                    tma_load_2d(&tmB, fb, st + C::OFF_B, ks * BK_BYTES, g.tn * BN);
+                    if (nbh > 0) bulk_load(st + C::OFF_SFB, sfb_row + ct0 * SF_CHUNK, sf_bytes, fb);
+                    if (C::BH == 2 && nbh > 1)
+                        bulk_load(st + C::OFF_SFB + SFA_BYTES, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
+                                  sf_bytes, fb);
+                }
+            };
+            // Static A side (the weights, in the decode form): the first
+            // STAGES stages' A tiles and scales are requested before the
+            // dependency wait, so they stream in while the previous kernel
+            // finishes; their B sides follow after it.
+            int pre_n = 0;
+            if (STREAM_K && p.a_static) {
+                Schedule<STREAM_K> pre(p);
+                Seg g;
+                while (pre_n < STAGES && pre.next(g)) {
+                    const int nbh = count_nbh(g);
+                    for (int ks = g.kb; ks < g.ke && pre_n < STAGES; ++ks, ++pre_n)
+                        issue(pre_n, g, ks, nbh, true, false, true);
+                }
+            }
             pdl_wait();
             Schedule<STREAM_K> sched(p);
             Seg sg;
@@ -518,33 +565,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             int issued = 0;
             bool ok = true;
             while (ok && sched.next(sg)) {
-                // scale row tiles of B that exist for this tile
-                const int rtb0 = (sg.tn * BN) / 128;
-                int nbh = 0;
-                for (int h = 0; h < C::BH; ++h)
-                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
-                const uint8_t* sfa_row = p.sfa + sg.tm * sf_row_bytes;
-                const uint8_t* sfb_row = p.sfb + rtb0 * sf_row_bytes;
-                const int ya = sg.tm * BM, yb = sg.tn * BN;
+                const int nbh = count_nbh(sg);
                 for (int ks = sg.kb; ks < sg.ke; ++ks) {
-                    const uint32_t fb = bar0 + 8u * stage;
-                    if (!wait_fast(bar0 + 8u * (STAGES + stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
-                        ok = false;
-                        break;
+                    if (issued < pre_n) {
+                        issue(stage, sg, ks, nbh, false, true, false);   // A side already requested
+                    } else {
+                        if (!wait_fast(bar0 + 8u * (STAGES + stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
+                            ok = false;
+                            break;
+                        }
+                        issue(stage, sg, ks, nbh, true, true, true);
                     }
-                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
-                    const int nch = MX ? nk / 2 : nk;
-                    const int ct0 = MX ? ks * 2 : ks * 4;   // first 512-byte scale chunk of the stage
-                    const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
-                    const uint32_t st = smem0 + stage * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(fb, A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
-                    tma_load_2d(&tmA, fb, st, ks * BK_BYTES, ya);
-                    tma_load_2d(&tmB, fb, st + C::OFF_B, ks * BK_BYTES, yb);
-                    bulk_load(st + C::OFF_SFA, sfa_row + ct0 * SF_CHUNK, sf_bytes, fb);
-                    if (nbh > 0) bulk_load(st + C::OFF_SFB, sfb_row + ct0 * SF_CHUNK, sf_bytes, fb);
-                    if (C::BH == 2 && nbh > 1)
-                        bulk_load(st + C::OFF_SFB + SFA_BYTES, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
-                                  sf_bytes, fb);
                     ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -1490,6 +1521,7 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.counters = nullptr;
     p.units = 0;
     p.sk_tiles = 0;
+    p.a_static = 0;
     p.max_seg = 0;
 }
 
@@ -1571,6 +1603,7 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     const DecodeSchedule d = decode_schedule(p.tiles_m, p.ks_total, dev.sm_count);
     const int G = d.G;
     p.sk_tiles = d.sk_tiles;
+    p.a_static = a.b_static ? 1 : 0;   // the weight operand B is the MMA A side here
     p.units = d.sk_tiles * p.ks_total;
     p.max_seg = d.max_seg;
     // the counters start at zero (caller's contract) and the kernel leaves

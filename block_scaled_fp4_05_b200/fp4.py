@@ -14,6 +14,7 @@ import torch
 NVFP4, MXFP4 = 0, 1
 ROWWISE, COLWISE = 0, 1
 GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE = 0, 1, 2
+GEMM_B_STATIC = 0x100   # flag: B / sB not written by a kernel still running on the stream
 
 FP4_OK = 0
 STATUS_NAMES = {
@@ -244,6 +245,11 @@ class BoundCall:
         st = self._f(*self._args)
         if st != FP4_OK:
             _check(st, self.name)
+
+    def on_stream(self, stream):
+        """The same call issued on another stream (the stream is the last
+        argument of every bound entry point)."""
+        return BoundCall(self.name, *self._args[:-1], _stream(stream))
 
 
 def bind_global_scale(x, gs_out, stream=None):

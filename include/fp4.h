@@ -82,7 +82,13 @@ typedef enum {
 typedef enum {
     FP4_GEMM_AUTO = 0,    /* decode kernel when M <= 16 and the workspace suffices, else prefill */
     FP4_GEMM_PREFILL = 1, /* persistent 128x256-tile tensor-core kernel */
-    FP4_GEMM_DECODE = 2   /* swap-AB, stream-K kernel for M <= 16 plus a split-K reduction */
+    FP4_GEMM_DECODE = 2,  /* swap-AB, stream-K kernel for M <= 16 plus a split-K reduction */
+    /* Flag, OR-ed into a kernel choice above: B and sB are not written by any
+     * kernel that may still be running on the stream when the GEMM starts
+     * (e.g. weights quantized ahead of time).  The decode kernel then requests
+     * its first weight tiles before waiting for the previous kernel to
+     * complete.  Without the flag no operand is read before that. */
+    FP4_GEMM_B_STATIC = 0x100
 } fp4_gemm_kernel;
 
 /* Version of this ABI (incremented on any signature or contract change). */
@@ -206,7 +212,8 @@ fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B
                     void* D, int64_t ldd, void* workspace, size_t ws_bytes,
                     fp4_stream_t stream);
 
-/* Same as fp4_gemm with an explicit kernel choice.  FP4_GEMM_DECODE needs
+/* Same as fp4_gemm with an explicit kernel choice (optionally OR-ed with
+ * FP4_GEMM_B_STATIC; other bits: FP4_ERR_INVALID_ARG).  FP4_GEMM_DECODE needs
  * M <= 16, N <= 524288 and a workspace of fp4_gemm_workspace_bytes bytes
  * (else FP4_ERR_UNSUPPORTED_SHAPE / FP4_ERR_INVALID_ARG). */
 fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, const void* B,

@@ -134,6 +134,40 @@ def test_decode_workspace_not_zeroed_is_reported():
     assert fp4.fp4_get_device_status() == 0
 
 
+@pytest.mark.parametrize("M", [1, 16])
+def test_dynamic_activation_then_decode_with_static_weights(orc, M):
+    # the chain a decode step runs: the activation is quantized with its own
+    # S_global (which also writes alpha) and the GEMM, launched right behind
+    # it with the weights marked static, requests weight tiles before the
+    # quantizer has finished; operands, scales and alpha of the activation
+    # must still be the quantizer's output
+    fmt, N, K = fp4.NVFP4, 38400, 2048   # 300 weight tiles: stream-K and whole tiles
+    A = synth.normal_bf16(M, K, seed=44, outlier_factor=100.0)
+    W = synth.normal_bf16(N, K, seed=44, tensor_id=1, sigma=0.02)
+    gW = orc.global_scale(W)
+    pW, sW = orc.quantize(fmt, 0, W, gs=gW)
+    Wd, sWd = to_dev_u8(pW), to_dev_u8(sW)
+    Ad = to_dev_bf16(A)
+    pA = torch.empty((M, K // 2), dtype=torch.uint8, device="cuda")
+    sA = torch.empty((fp4.fp4_scale_bytes(fmt, M, K),), dtype=torch.uint8, device="cuda")
+    gA = torch.empty(1, dtype=torch.float32, device="cuda")
+    alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros((fp4.fp4_gemm_workspace_bytes(fmt, M, N, K),), dtype=torch.uint8, device="cuda")
+    D = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    for _ in range(3):   # repeated back to back: each pair reads the previous pair's buffers
+        pA.fill_(0xFF)
+        fp4.fp4_quantize_dynamic(Ad, pA, sA, gA, to_dev_f32(gW), alpha)
+        fp4.fp4_gemm(fmt, pA, sA, Wd, sWd, M, N, K, alpha, D, ws,
+                     kernel=fp4.GEMM_DECODE | fp4.GEMM_B_STATIC)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    g = orc.global_scale(A)
+    qA, sqA = orc.quantize(fmt, 0, A, gs=g)
+    D_orc, S = orc.gemm(fmt, qA, sqA, pW, sW, alpha=float(np.float32(g) * np.float32(gW)))
+    assert_gemm_close(bf16_dev_to_f64(D), D_orc, S, "dynamic + decode, static weights")
+
+
 def test_k_zero_and_empty():
     A = torch.empty((4, 0), dtype=torch.uint8, device="cuda")
     B = torch.empty((8, 0), dtype=torch.uint8, device="cuda")
