@@ -179,18 +179,15 @@ class SquareWorkload(Workload):
     """Quantize A and B (rowwise, along K) and D = A_hat B_hat^T, M=N=K=n."""
 
     def __init__(self, fmt, n, dev, sets=4, stream=None):
-        # quantize A and quantize B are independent: B runs on a second stream
-        # (a parallel branch in the captured graph) and the GEMM waits for both
         self.stream = stream if stream is not None else torch.cuda.current_stream()
-        self.stream2 = torch.cuda.Stream(device=dev)
-        self.fork = torch.cuda.Event()
-        self.join = torch.cuda.Event()
         self.fmt, self.n = fmt, n
         self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
         A, B = synth.square(n)
         self.host = (A, B)
-        self.kernels = ["quantize_A", "quantize_B", "gemm"] if fmt == fp4.MXFP4 else \
-            ["global_scales", "quantize_A", "quantize_B", "gemm"]
+        # A and B are quantized by one batched launch (one persistent grid over
+        # the tiles of both), then the GEMM
+        self.kernels = ["quantize", "gemm"] if fmt == fp4.MXFP4 else \
+            ["global_scales", "quantize", "gemm"]
         self.calls = []
         self.bufs = []
         for s in range(sets):
@@ -207,55 +204,22 @@ class SquareWorkload(Workload):
                                fp4.bind_alpha(gA, gB, al, stream)])
             else:
                 gA = gB = al = None
-            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Ad, pA, sA, gA, stream)])
-            groups.append([fp4.bind_quantize(fmt, fp4.ROWWISE, Bd, pB, sB, gB, self.stream2)])
+            groups.append([fp4.bind_quantize_batch(fmt, [(Ad, pA, sA, gA), (Bd, pB, sB, gB)], stream)])
             groups.append([fp4.bind_gemm(fmt, pA, sA, pB, sB, n, n, n, al, D, None, fp4.GEMM_PREFILL,
                                          stream)])
             self.calls.append(groups)
             self.bufs.append((Ad, Bd, pA, sA, pB, sB, D, gA, gB, al))
-        kb = fp4.block_size(fmt)
         qbytes = n * n * 2 + n * n // 2 + fp4.fp4_scale_bytes(fmt, n, n)
-        self.work = {"quantize_A": qbytes, "quantize_B": qbytes, "gemm": 2.0 * n ** 3,
-                     "global_scales": 2.0 * n * n * 2}
-        self.bound = {"quantize_A": "hbm", "quantize_B": "hbm", "gemm": "tensor",
-                      "global_scales": "hbm"}
+        self.work = {"quantize": 2 * qbytes, "gemm": 2.0 * n ** 3, "global_scales": 2.0 * n * n * 2}
+        self.bound = {"quantize": "hbm", "gemm": "tensor", "global_scales": "hbm"}
         self.flops = 2.0 * n ** 3
-        self.launches_per_step = 3 if fmt == fp4.MXFP4 else 3 + 2 * 2 + 1
+        self.launches_per_step = 2 if fmt == fp4.MXFP4 else 2 + 2 * 2 + 1
         self.dominant = "gemm"
         self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
             sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
-        del kb
 
     def value(self, sec_per_step):
         return self.flops / sec_per_step / 1e12
-
-    def step(self, i, ev=None):
-        calls = self.calls[i % len(self.calls)]
-        names = self.kernels
-        qa, qb = names.index("quantize_A"), names.index("quantize_B")
-        for k, group in enumerate(calls):
-            if k == qb:
-                continue
-            if k == qa:
-                # fork: B's quantization on the second stream, concurrently
-                self.fork.record(self.stream)
-                self.stream2.wait_event(self.fork)
-                with torch.cuda.stream(self.stream2):
-                    if ev is not None:
-                        ev[qb][0].record(self.stream2)
-                    for c in calls[qb]:
-                        c()
-                    if ev is not None:
-                        ev[qb][1].record(self.stream2)
-                self.join.record(self.stream2)
-            if ev is not None:
-                ev[k][0].record(self.stream)
-            for c in group:
-                c()
-            if ev is not None:
-                ev[k][1].record(self.stream)
-            if k == qa:
-                self.stream.wait_event(self.join)
 
     def e2e_setup(self, dev):
         A, B = self.host
@@ -274,8 +238,9 @@ class SquareWorkload(Workload):
             fp4.fp4_alpha_from_global_scales(gA, gB, al)
         else:
             gA = gB = al = None
-        pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, gA)
-        pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, gB)
+        pA, sA = _qbufs(fmt, n, n, dev)
+        pB, sB = _qbufs(fmt, n, n, dev)
+        fp4.fp4_quantize_batch(fmt, [(Ad, pA, sA, gA), (Bd, pB, sB, gB)])
         D = fp4.gemm(fmt, pA, sA, pB, sB, n, alpha=al, kernel=fp4.GEMM_PREFILL)
         self.hD.copy_(D, non_blocking=True)
 

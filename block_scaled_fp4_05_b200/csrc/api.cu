@@ -153,6 +153,46 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
         fmt == FP4_NVFP4 ? global_scale : nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* descs,
+                              fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_fmt(fmt) || n < 0 || (n > 0 && !descs)) return FP4_ERR_INVALID_ARG;
+    const int kb = fp4::block_size(fmt);
+    int work = 0;
+    for (int i = 0; i < n; ++i) {
+        const fp4_quantize_desc& d = descs[i];
+        if (d.rows < 0 || d.cols < 0 || d.ld < d.cols) return FP4_ERR_INVALID_ARG;
+        if (d.rows == 0 || d.cols == 0) continue;
+        ++work;
+        if (!d.in_bf16 || !d.packed_out || !d.scales_out) return FP4_ERR_INVALID_ARG;
+        if (fmt == FP4_NVFP4 && !d.global_scale) return FP4_ERR_INVALID_ARG;
+        if (d.cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (d.rows >= kMaxRows || d.cols >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (d.ld % 8 != 0 || !aligned16(d.in_bf16) || !aligned16(d.packed_out) || !aligned16(d.scales_out))
+            return FP4_ERR_MISALIGNED;
+        if (d.global_scale && (reinterpret_cast<uintptr_t>(d.global_scale) & 3u)) return FP4_ERR_MISALIGNED;
+    }
+    if (work == 0) return FP4_OK;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    fp4::RowwiseDesc local[16];
+    for (int i0 = 0; i0 < n; i0 += 16) {
+        const int m = n - i0 < 16 ? n - i0 : 16;
+        for (int i = 0; i < m; ++i) {
+            const fp4_quantize_desc& d = descs[i0 + i];
+            local[i] = {static_cast<const uint16_t*>(d.in_bf16), d.rows, d.cols, d.ld,
+                        static_cast<uint8_t*>(d.packed_out), static_cast<uint8_t*>(d.scales_out),
+                        fmt == FP4_NVFP4 ? d.global_scale : nullptr};
+        }
+        st = from_cuda(fp4::launch_quantize_rowwise_batch((int)fmt, m, local,
+                                                          reinterpret_cast<cudaStream_t>(stream)));
+        if (st != FP4_OK) return st;
+    }
+    return FP4_OK;
+}
+
 fp4_status fp4_quantize_dynamic(fp4_format fmt, const void* in_bf16, int64_t rows, int64_t cols,
                                 int64_t ld, void* packed_out, void* scales_out, float* gs_out,
                                 const float* other_gs, float* alpha_out, fp4_stream_t stream)

@@ -32,6 +32,15 @@ cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t col
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
                             cudaStream_t s);
+// Rowwise quantization of n tensors, batched into persistent launches.
+struct RowwiseDesc {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    uint8_t* packed;
+    uint8_t* scales;
+    const float* gs;   // NVFP4 S_global, NULL for MXFP4
+};
+cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s);
 
 // gemm.cu
 struct GemmArgs {

@@ -26,6 +26,7 @@ namespace fp4 {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kMaxBatch = 8;   // tensors per batched launch
 
 // Lets a kernel launched after this one with programmatic stream
 // serialization (the GEMMs) start its set-up; it still waits for this
@@ -178,20 +179,48 @@ __device__ __forceinline__ void rowwise_tile(const uint16_t* __restrict__ x, int
     }
 }
 
+// The tile list of a batch of tensors: tile t belongs to tensor k with
+// tile_begin[k] <= t < tile_begin[k+1]; within a tensor, column tiles run
+// fastest.  Used by both rowwise kernels (with their own tile widths).
+struct RowBatch {
+    int n;
+    int64_t tile_begin[kMaxBatch + 1];   // prefix sums of the tensors' tile counts
+    const uint16_t* x[kMaxBatch];
+    int64_t rows[kMaxBatch], cols[kMaxBatch], ld[kMaxBatch];
+    uint8_t* packed[kMaxBatch];
+    uint8_t* scales[kMaxBatch];
+    const float* gs[kMaxBatch];
+};
+
+__device__ __forceinline__ void locate_tile(const RowBatch& b, int64_t t, int64_t tile_c, int& k,
+                                            int64_t& rt, int64_t& ct)
+{
+    k = 0;
+    while (t >= b.tile_begin[k + 1]) ++k;
+    const int64_t local = t - b.tile_begin[k];
+    const int64_t nct = (b.cols[k] + tile_c - 1) / tile_c;
+    rt = local / nct;
+    ct = local - rt * nct;
+}
+
+// One CTA per 128-row x 4-block tile: grid = all tiles of the batch.
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
-quantize_rowwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-                        uint8_t* __restrict__ packed, uint8_t* __restrict__ scales,
-                        const float* __restrict__ gs_ptr)
+quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
 {
     __shared__ __align__(16) uint8_t s_tile[512];
     pdl_trigger();
+    constexpr int TILE_C = 4 * (FMT == kMx ? 32 : 16);
+    int k;
+    int64_t rt, ct;
+    locate_tile(b, blockIdx.x, TILE_C, k, rt, ct);
     float gs = 1.0f, denom = 6.0f;
     if (FMT == kNv) {
-        gs = __ldg(gs_ptr);
+        gs = __ldg(b.gs[k]);
         denom = __fmul_rn(6.0f, gs);
     }
-    rowwise_tile<FMT>(x, rows, cols, ld, packed, scales, blockIdx.y, blockIdx.x, gs, denom, s_tile);
+    rowwise_tile<FMT>(b.x[k], b.rows[k], b.cols[k], b.ld[k], b.packed[k], b.scales[k], rt, ct, gs, denom,
+                      s_tile);
 }
 
 // ---------------------------------------------------------------------------
@@ -569,6 +598,42 @@ cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t col
     return e;
 }
 
+// One launch over the tiles of up to kMaxBatch tensors.  (A persistent
+// variant that streamed the tiles through a cp.async ring in shared memory
+// was measured slower for both formats: one CTA per tile, many of them
+// resident, keeps more loads in flight.)
+cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s)
+{
+    const int64_t tile_c = 4 * block_size(fmt);
+    for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
+        RowBatch b = {};
+        b.n = 0;
+        b.tile_begin[0] = 0;
+        for (int i = i0; i < n && i < i0 + kMaxBatch; ++i) {
+            if (d[i].rows == 0 || d[i].cols == 0) continue;
+            const int j = b.n++;
+            b.x[j] = d[i].x;
+            b.rows[j] = d[i].rows;
+            b.cols[j] = d[i].cols;
+            b.ld[j] = d[i].ld;
+            b.packed[j] = d[i].packed;
+            b.scales[j] = d[i].scales;
+            b.gs[j] = d[i].gs;
+            b.tile_begin[j + 1] = b.tile_begin[j] + ((d[i].rows + 127) / 128) * ((d[i].cols + tile_c - 1) / tile_c);
+        }
+        if (b.n == 0) continue;
+        const int64_t tiles = b.tile_begin[b.n];
+        if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
+        if (fmt == kNv)
+            quantize_rowwise_tiles_kernel<kNv><<<(unsigned)tiles, kThreads, 0, s>>>(b);
+        else
+            quantize_rowwise_tiles_kernel<kMx><<<(unsigned)tiles, kThreads, 0, s>>>(b);
+        const cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
                             cudaStream_t s)
@@ -576,11 +641,8 @@ cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, 
     if (rows == 0 || cols == 0) return cudaSuccess;
     const int kb = block_size(fmt);
     if (axis == 0) {
-        dim3 grid((unsigned)(cols / (4 * kb)), (unsigned)((rows + 127) / 128));
-        if (fmt == kNv)
-            quantize_rowwise_kernel<kNv><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
-        else
-            quantize_rowwise_kernel<kMx><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+        const RowwiseDesc d = {x, rows, cols, ld, packed, scales, gs};
+        return launch_quantize_rowwise_batch(fmt, 1, &d, s);
     } else {
         dim3 grid((unsigned)(rows / (4 * kb)), (unsigned)((cols + 127) / 128));
         if (fmt == kNv)

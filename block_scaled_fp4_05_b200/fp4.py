@@ -62,6 +62,8 @@ def lib():
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
+        L.fp4_quantize_batch.restype = c.c_int
+        L.fp4_quantize_batch.argtypes = [c.c_int, c.c_int, P, st]
         L.fp4_quantize_dynamic.restype = c.c_int
         L.fp4_quantize_dynamic.argtypes = [c.c_int, P, i64, i64, i64, P, P, P, P, P, st]
         L.fp4_alpha_from_global_scales.restype = c.c_int
@@ -148,6 +150,39 @@ def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream
                               _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
                               _dptr(global_scale, "global_scale"), _stream(stream)),
            "fp4_quantize")
+
+
+class QuantizeDesc(ctypes.Structure):
+    """fp4_quantize_desc of include/fp4.h."""
+    _fields_ = [("in_bf16", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ld", ctypes.c_int64), ("packed_out", ctypes.c_void_p), ("scales_out", ctypes.c_void_p),
+                ("global_scale", ctypes.c_void_p)]
+
+
+def _quantize_descs(items):
+    arr = (QuantizeDesc * max(1, len(items)))()
+    for i, (x, packed_out, scales_out, gs) in enumerate(items):
+        assert x.dtype == torch.bfloat16
+        arr[i] = QuantizeDesc(_dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                              _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
+                              _dptr(gs, "global_scale"))
+    return arr
+
+
+def fp4_quantize_batch(fmt, items, stream=None):
+    """Rowwise quantization of several tensors in one launch; items are
+    (x, packed_out, scales_out, global_scale or None) tuples."""
+    arr = _quantize_descs(items)
+    _check(lib().fp4_quantize_batch(int(fmt), len(items), ctypes.cast(arr, ctypes.c_void_p),
+                                    _stream(stream)), "fp4_quantize_batch")
+
+
+def bind_quantize_batch(fmt, items, stream=None):
+    arr = _quantize_descs(items)
+    call = BoundCall("fp4_quantize_batch", int(fmt), len(items), ctypes.cast(arr, ctypes.c_void_p),
+                     _stream(stream))
+    call.keep = arr   # the descriptor array must outlive the bound call
+    return call
 
 
 def fp4_quantize_dynamic(x, packed_out, scales_out, gs_out, other_gs=None, alpha_out=None,
@@ -249,7 +284,10 @@ class BoundCall:
     def on_stream(self, stream):
         """The same call issued on another stream (the stream is the last
         argument of every bound entry point)."""
-        return BoundCall(self.name, *self._args[:-1], _stream(stream))
+        c = BoundCall(self.name, *self._args[:-1], _stream(stream))
+        if hasattr(self, "keep"):
+            c.keep = self.keep
+        return c
 
 
 def bind_global_scale(x, gs_out, stream=None):

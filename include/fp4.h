@@ -81,7 +81,7 @@ typedef enum {
 
 typedef enum {
     FP4_GEMM_AUTO = 0,    /* decode kernel when M <= 16 and the workspace suffices, else prefill */
-    FP4_GEMM_PREFILL = 1, /* persistent 128x256-tile tensor-core kernel */
+    FP4_GEMM_PREFILL = 1, /* persistent CTA-pair tensor-core kernel, 256x256 tiles */
     FP4_GEMM_DECODE = 2,  /* swap-AB, stream-K kernel for M <= 16 plus a split-K reduction */
     /* Flag, OR-ed into a kernel choice above: B and sB are not written by any
      * kernel that may still be running on the stream when the GEMM starts
@@ -154,14 +154,38 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
                         const float* global_scale, fp4_stream_t stream);
 
 /*
+ * Rowwise quantization of several tensors in one launch (e.g. both GEMM
+ * operands of a step), each exactly as fp4_quantize(fmt, FP4_ROWWISE, ...)
+ * with its own sizes, buffers and S_global.  One launch covers the 128-row
+ * tiles of up to 8 tensors (more are split into several launches), so small
+ * tensors do not each pay a launch and a partial last wave.  Every
+ * descriptor is validated before anything is launched; a failing one makes
+ * the call return its status having launched nothing.
+ *   n     : number of descriptors (>= 0)
+ *   descs : host array of n descriptors
+ */
+typedef struct {
+    const void* in_bf16;        /* device, rows x cols, leading dimension ld (elements) */
+    int64_t rows, cols, ld;
+    void* packed_out;           /* device, rows x cols/2 bytes */
+    void* scales_out;           /* device, fp4_scale_bytes(fmt, rows, cols) bytes */
+    const float* global_scale;  /* device S_global (NVFP4, required); NULL for MXFP4 */
+} fp4_quantize_desc;
+
+fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* descs,
+                              fp4_stream_t stream);
+
+/*
  * Dynamic NVFP4 quantization of a small tensor (e.g. the few rows of a decode
  * activation) in a single launch: S_global of the tensor (as
  * fp4_compute_global_scale), then the rowwise quantization with it (as
  * fp4_quantize), and optionally alpha = S_global * (*other_gs) (as
  * fp4_alpha_from_global_scales with the other operand's scale).  Results are
- * identical to those three calls.  One cluster of 8 CTAs does the work, so it
- * suits tensors of up to a few hundred thousand elements; larger tensors are
- * correct but use only 8 SMs.
+ * identical to those three calls.  One cluster of 16 CTAs (8 where the device
+ * cannot place 16) holds the tensor in registers between the amax and the
+ * quantization; a tensor above that capacity (65536 16-byte chunks, i.e.
+ * 1 MiB of BF16, with 16 CTAs) is handled inside the same call by the
+ * separate amax, quantize and alpha kernels.
  *   fmt      : FP4_NVFP4 only (MXFP4 needs no per-tensor scale: use
  *              fp4_quantize); else FP4_ERR_INVALID_ARG
  *   in_bf16  : device, rows x cols (ld), cols % 64 == 0, rows, cols > 0

@@ -75,3 +75,26 @@ def test_gemm_host_checks_without_gpu():
         assert L.fp4_compute_global_scale(A16, 4, 8, 8, A16, None) == 6
     assert L.fp4_compute_global_scale(A16, 4, 12, 12, A16, None) == 2
     assert L.fp4_alpha_from_global_scales(None, A16, A16, None) == 1
+
+
+def test_quantize_batch_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    D = fp4.QuantizeDesc
+
+    def call(fmt, descs):
+        arr = (D * max(1, len(descs)))(*descs)
+        return L.fp4_quantize_batch(fmt, len(descs), ctypes.cast(arr, P), None)
+
+    good = D(1 << 20, 128, 512, 512, 1 << 20, 1 << 20, 1 << 20)
+    assert call(5, [good]) == 1                                          # bad format
+    assert L.fp4_quantize_batch(0, -1, None, None) == 1                  # negative count
+    assert L.fp4_quantize_batch(0, 2, None, None) == 1                   # NULL array
+    assert call(0, [good, D(1 << 20, 128, 480, 480, 1 << 20, 1 << 20, 1 << 20)]) == 2   # cols % 64
+    assert call(1, [D(1 << 20, 128, 192, 192, 1 << 20, 1 << 20, None)]) == 2           # cols % 128 (MX)
+    assert call(0, [D(1 << 20, 128, 512, 512, 1 << 20, 1 << 20, None)]) == 1           # NV without S_global
+    assert call(0, [D((1 << 20) + 2, 128, 512, 512, 1 << 20, 1 << 20, 1 << 20)]) == 3  # misaligned
+    assert call(0, [D(0, 0, 512, 512, 0, 0, 0)]) == 0                                   # empty only: no-op
+    assert L.fp4_quantize_batch(0, 0, None, None) == 0
+    if not torch.cuda.is_available():
+        assert call(0, [good]) == 6                                      # valid, but no device here

@@ -47,7 +47,8 @@ def test_tiny_config(orc, fmt, axis):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("shape", [(1, 512), (3, 256), (129, 384), (200, 1024), (517, 2048)])
+@pytest.mark.parametrize("shape", [(1, 512), (3, 256), (129, 384), (200, 1024), (517, 2048),
+                                   (33, 320), (130, 64)])   # NVFP4 only: a 64-column last tile
 def test_rowwise_ragged_rows(orc, fmt, shape):
     if shape[1] % (4 * fp4.block_size(fmt)):
         pytest.skip("length not a multiple of 4 blocks")
@@ -209,3 +210,30 @@ def test_dynamic_quantize_all_zero_and_rejects_mx():
                                         ctypes.c_void_p(p.data_ptr()), ctypes.c_void_p(s.data_ptr()),
                                         ctypes.c_void_p(gs.data_ptr()), None, None, None)
     assert st == 1
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_batch_matches_oracle_per_tensor(orc, fmt):
+    # ten tensors in one call (more than one launch's eight), ragged row
+    # counts, one empty; each must equal its own fp4_quantize result
+    shapes = [(517, 2048), (1, 512), (128, 256), (0, 256), (200, 1024), (3, 128), (129, 384),
+              (64, 4096), (1000, 128), (7, 640)]
+    items, expect = [], []
+    for i, (r, c) in enumerate(shapes):
+        x = synth.normal_bf16(max(r, 1), c, seed=50 + i, outlier_factor=60.0, zero_frac=0.02)[:r]
+        gs = orc.global_scale(x) if (fmt == fp4.NVFP4 and r > 0) else 1.0
+        packed = Guarded(max(1, r * c // 2))
+        scales = Guarded(max(1, fp4.fp4_scale_bytes(fmt, r, c)), fill=0x5A)
+        xd = to_dev_bf16(x) if r > 0 else torch.empty((0, c), dtype=torch.bfloat16, device="cuda")
+        items.append((xd, packed.view, scales.view, to_dev_f32(gs) if fmt == fp4.NVFP4 else None))
+        expect.append((x, gs, packed, scales))
+    fp4.fp4_quantize_batch(fmt, items)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    for (r, c), (x, gs, packed, scales) in zip(shapes, expect):
+        assert packed.guards_intact() and scales.guards_intact()
+        if r == 0:
+            continue
+        p_orc, s_orc = orc.quantize(fmt, fp4.ROWWISE, x, gs=gs)
+        assert np.array_equal(packed.view.cpu().numpy().reshape(r, c // 2), p_orc), (r, c)
+        assert np.array_equal(scales.view.cpu().numpy(), s_orc), (r, c)
