@@ -933,10 +933,29 @@ struct PairCfg {
     static constexpr int SF_COLS = SFA_COLS + 8 * NCH;
     static constexpr int TMEM_COLS = 512;
     static constexpr int NBARS = 5 * STAGES + 4;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 512;
+    // epilogue staging: per epilogue warp one 32-row x 32-column BF16 block
+    // (64-byte rows, 64-byte swizzle) that a TMA store writes to D
+    static constexpr int EPI_BLOCK = 32 * 64;
+    static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
+    static constexpr int OFF_BARS = OFF_EPI + 4 * EPI_BLOCK;
+    static constexpr int SMEM = OFF_BARS + 1024 + 512;
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
     static_assert(NBARS * 8 + 8 <= 512, "barrier area");
+    static_assert(SMEM <= 232448, "shared memory per CTA");
 };
+
+// 2-D TMA store of a shared-memory box to global memory (bulk-group
+// completion), and the waits on this thread's bulk groups.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t cluster_rank()
 {
@@ -1034,13 +1053,13 @@ __device__ __forceinline__ void spin_ns(uint64_t ns)
 template <int STAGES, bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Params p)
+                     const __grid_constant__ CUtensorMap tmD, const Params p)
 {
     using C = PairCfg<STAGES, MX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
     // [0,S) full (leader), [S,2S) empty, [2S,3S) sf_full, [3S,4S) sf_ready (leader),
     // [4S] acc_full, [4S+1] acc_empty (leader), [4S+2] drain
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
@@ -1240,20 +1259,36 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 else
                     mbar_arrive_cluster_relaxed(acc_empty_leader);
             }
+            // D through shared memory: the warp's 32 rows x 32 columns at a
+            // time go to its staging block (64-byte rows; 16-byte chunk j of
+            // row r at chunk j ^ ((r >> 1) & 3), the 64-byte swizzle), then
+            // one lane stores the block with TMA, coalesced and clipped to D.
             const int tm = t % p.tiles_m, tn = t / p.tiles_m;
-            const int64_t gm = (int64_t)(tm * 2 + (int)rank) * BM + row;
-            if (gm < p.rows_a) {
-                uint16_t* drow = p.D + gm * p.ldd + (int64_t)tn * PAIR_BN;
-                const int ncols = p.rows_b - tn * PAIR_BN;
+            const int y0 = (tm * 2 + (int)rank) * BM + q * 32;
+            const uint32_t blk = smem0 + C::OFF_EPI + q * C::EPI_BLOCK;
+            const uint32_t my_row = blk + lane * 64;
+            const int sw = (lane >> 1) & 3;
+            if (y0 < p.rows_a) {
 #pragma unroll
-                for (int i = 0; i < PAIR_BN / 8; ++i)
-                    if (i * 8 < ncols)
-                        *reinterpret_cast<uint4*>(drow + i * 8) =
-                            make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
-                                       packed[4 * i + 3]);
+                for (int c = 0; c < PAIR_BN / 32; ++c) {
+                    const int x0 = tn * PAIR_BN + c * 32;
+                    if (x0 >= p.rows_b) break;
+                    if (lane == 0) bulk_wait_read_all();   // the block's previous store has read it
+                    __syncwarp();
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(my_row + ((j ^ sw) << 4)),
+                                     "r"(packed[c * 16 + 4 * j]), "r"(packed[c * 16 + 4 * j + 1]),
+                                     "r"(packed[c * 16 + 4 * j + 2]), "r"(packed[c * 16 + 4 * j + 3])
+                                     : "memory");
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&tmD, blk, x0, y0);
+                }
             }
             acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait_all();   // every store of D has completed
     } else {
         // ---------------- scale staging (warps 6..9, both CTAs) ----------------
         const uint32_t tq = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
@@ -1371,6 +1406,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder()
 
 // 2-D map over a packed operand [rows x row_bytes] (uint8), box 128 bytes x
 // box_rows, 128-byte swizzle, zero fill out of bounds.
+// D [rows x cols] BF16 with leading dimension ld (elements), stored by the
+// pair kernel's epilogue in 32 x 32 boxes with the 64-byte swizzle.
+bool make_map_d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld)
+{
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_rows)
 {
     auto enc = encoder();
@@ -1526,8 +1576,8 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
 }
 
 template <int STAGES, bool MX>
-cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
-                               int grid, cudaStream_t s)
+cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
+                               const Params& p, int grid, cudaStream_t s)
 {
     using C = PairCfg<STAGES, MX>;
     auto kern = fp4_gemm_pair_kernel<STAGES, MX>;
@@ -1561,7 +1611,7 @@ cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, con
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p);
     if (e != cudaSuccess) set_last_error("pair GEMM kernel launch", e);
     return e;
 }
@@ -1571,8 +1621,9 @@ constexpr int PAIR_STAGES_MX = 6;   // 35 KB per stage
 
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
 {
-    CUtensorMap ta, tb;
-    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PAIR_BHALF)) {
+    CUtensorMap ta, tb, td;
+    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PAIR_BHALF) ||
+        !make_map_d(&td, a.D, a.M, a.N, a.ldd)) {
         set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return cudaErrorInvalidValue;
     }
@@ -1583,8 +1634,8 @@ cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaSt
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     const int64_t max_pairs = dev.sm_count / 2;
     const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
-    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true>(ta, tb, p, grid, s);
-    return launch_pair_kernel<PAIR_STAGES_NV, false>(ta, tb, p, grid, s);
+    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true>(ta, tb, td, p, grid, s);
+    return launch_pair_kernel<PAIR_STAGES_NV, false>(ta, tb, td, p, grid, s);
 }
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
