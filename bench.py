@@ -347,13 +347,14 @@ class QuantWorkload(Workload):
     def __init__(self, fmt, axis, rows, cols, dev, stream=None):
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.fmt, self.axis = fmt, axis
-        self.name = "%s %s quantize %dx%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4",
+        self.name = "%s %s quantize %dx%d" % ({fp4.NVFP4: "NVFP4", fp4.MXFP4: "MXFP4",
+                                               fp4.P1E8: "E8M0/16 under S_global"}[fmt],
                                               "rowwise" if axis == fp4.ROWWISE else "colwise",
                                               rows, cols)
         x = synth.quant_sweep(rows, cols)
         self.host = (x,)
         xd = _dev_bf16(x, dev)
-        gs = fp4.global_scale(xd) if fmt == fp4.NVFP4 else None
+        gs = fp4.global_scale(xd) if fmt != fp4.MXFP4 else None
         out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
         p, s = _qbufs(fmt, out_rows, K, dev)
         self.calls = [[[fp4.bind_quantize(fmt, axis, xd, p, s, gs, stream)]]]
@@ -424,14 +425,14 @@ def make_workload(name, dev, stream):
     if name.startswith("quant_"):
         _, shape, f, ax = name.split("_")
         rows, cols = (16384, 16384) if shape == "16384" else (8192, 28672)
-        return QuantWorkload(fp4.NVFP4 if f == "nv" else fp4.MXFP4,
-                             fp4.ROWWISE if ax == "row" else fp4.COLWISE, rows, cols, dev, stream=stream)
+        fmt = {"nv": fp4.NVFP4, "mx": fp4.MXFP4, "p1e8": fp4.P1E8}[f]
+        return QuantWorkload(fmt, fp4.ROWWISE if ax == "row" else fp4.COLWISE, rows, cols, dev, stream=stream)
     raise SystemExit("unknown workload %r" % name)
 
 
 WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
              "prefill_down"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
-                                for f in ("nv", "mx") for a in ("row", "col")]
+                                for f in ("nv", "mx", "p1e8") for a in ("row", "col")]
 
 
 # ---------------------------------------------------------------------------

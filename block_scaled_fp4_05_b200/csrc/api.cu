@@ -46,7 +46,9 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Formats of the GEMM entry points, and the quantizer's (which adds P1E8).
 bool valid_fmt(fp4_format f) { return f == FP4_NVFP4 || f == FP4_MXFP4; }
+bool valid_quant_fmt(fp4_format f) { return valid_fmt(f) || f == FP4_P1E8; }
 
 fp4_status from_cuda(cudaError_t e)
 {
@@ -101,7 +103,7 @@ size_t fp4_packed_bytes(int64_t rows, int64_t k)
 
 size_t fp4_scale_bytes(fp4_format fmt, int64_t rows, int64_t k)
 {
-    if (!valid_fmt(fmt) || rows <= 0 || k <= 0) return 0;
+    if (!valid_quant_fmt(fmt) || rows <= 0 || k <= 0) return 0;
     const int64_t nsc = k / fp4::block_size(fmt);
     return (size_t)((rows + 127) / 128) * (size_t)((nsc + 3) / 4) * 512u;
 }
@@ -128,11 +130,11 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
                         const float* global_scale, fp4_stream_t stream)
 {
     fp4::g_last_error[0] = 0;
-    if (!valid_fmt(fmt) || (axis != FP4_ROWWISE && axis != FP4_COLWISE)) return FP4_ERR_INVALID_ARG;
+    if (!valid_quant_fmt(fmt) || (axis != FP4_ROWWISE && axis != FP4_COLWISE)) return FP4_ERR_INVALID_ARG;
     if (rows < 0 || cols < 0 || ld < cols) return FP4_ERR_INVALID_ARG;
     if (rows == 0 || cols == 0) return FP4_OK;
     if (!in_bf16 || !packed_out || !scales_out) return FP4_ERR_INVALID_ARG;
-    if (fmt == FP4_NVFP4 && !global_scale) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && !global_scale) return FP4_ERR_INVALID_ARG;
     const int kb = fp4::block_size(fmt);
     if (axis == FP4_ROWWISE) {
         if (cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
@@ -150,14 +152,14 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
     return from_cuda(fp4::launch_quantize(
         (int)fmt, (int)axis, static_cast<const uint16_t*>(in_bf16), rows, cols, ld,
         static_cast<uint8_t*>(packed_out), static_cast<uint8_t*>(scales_out),
-        fmt == FP4_NVFP4 ? global_scale : nullptr, reinterpret_cast<cudaStream_t>(stream)));
+        fmt != FP4_MXFP4 ? global_scale : nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* descs,
                               fp4_stream_t stream)
 {
     fp4::g_last_error[0] = 0;
-    if (!valid_fmt(fmt) || n < 0 || (n > 0 && !descs)) return FP4_ERR_INVALID_ARG;
+    if (!valid_quant_fmt(fmt) || n < 0 || (n > 0 && !descs)) return FP4_ERR_INVALID_ARG;
     const int kb = fp4::block_size(fmt);
     int work = 0;
     for (int i = 0; i < n; ++i) {
@@ -166,7 +168,7 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
         if (d.rows == 0 || d.cols == 0) continue;
         ++work;
         if (!d.in_bf16 || !d.packed_out || !d.scales_out) return FP4_ERR_INVALID_ARG;
-        if (fmt == FP4_NVFP4 && !d.global_scale) return FP4_ERR_INVALID_ARG;
+        if (fmt != FP4_MXFP4 && !d.global_scale) return FP4_ERR_INVALID_ARG;
         if (d.cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
         if (d.rows >= kMaxRows || d.cols >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
         if (d.ld % 8 != 0 || !aligned16(d.in_bf16) || !aligned16(d.packed_out) || !aligned16(d.scales_out))
@@ -184,7 +186,7 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
             const fp4_quantize_desc& d = descs[i0 + i];
             local[i] = {static_cast<const uint16_t*>(d.in_bf16), d.rows, d.cols, d.ld,
                         static_cast<uint8_t*>(d.packed_out), static_cast<uint8_t*>(d.scales_out),
-                        fmt == FP4_NVFP4 ? d.global_scale : nullptr};
+                        fmt != FP4_MXFP4 ? d.global_scale : nullptr};
         }
         st = from_cuda(fp4::launch_quantize_rowwise_batch((int)fmt, m, local,
                                                           reinterpret_cast<cudaStream_t>(stream)));

@@ -11,6 +11,7 @@ namespace fp4 {
 
 constexpr int kNv = 0;
 constexpr int kMx = 1;
+constexpr int kP1 = 2;   // 16-element blocks, E8M0 scale under S_global
 
 inline int block_size(int fmt) { return fmt == kMx ? 32 : 16; }
 

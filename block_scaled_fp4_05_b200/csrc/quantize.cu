@@ -1,5 +1,6 @@
-// Block quantizer kernels: BF16 -> E2M1 codes + per-block scales (NVFP4 /
-// MXFP4), the per-tensor amax for S_global, and alpha = gsA * gsB.
+// Block quantizer kernels: BF16 -> E2M1 codes + per-block scales (NVFP4,
+// MXFP4, and 16-element blocks with E8M0 scales under S_global), the
+// per-tensor amax for S_global, and alpha = gsA * gsB.
 //
 // Method: "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell",
 // "1. The Dual-Level Mathematical Formulation" (S_global, S_block,j, q_i) and
@@ -86,6 +87,16 @@ __device__ __forceinline__ uint32_t block_scale(uint32_t amax_bits, float gs, fl
             e = Eb - 129 + ((amax_bits & 0x7F) > 64 ? 1 : 0);
         }
         *inv = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+        return (uint32_t)(e + 127);
+    } else if (FMT == kP1) {
+        // e = ceil(log2(max(amax / (6 * S_global), 1e-8))) with the ratio
+        // formed in FP32; for a = f * 2^E (a is normal), e = E when f == 1,
+        // else E + 1; capped at 127.  S_block = 2^e, eff = S_block * S_global.
+        const float a = fmaxf(__fdiv_rn(amax, denom), 1e-8f);
+        const uint32_t ab = __float_as_uint(a);
+        const int e = min((int)(ab >> 23) - 127 + ((ab & 0x7FFFFFu) ? 1 : 0), 127);
+        const float eff = __fmul_rn(__uint_as_float((uint32_t)(e + 127) << 23), gs);
+        *inv = (eff == 0.0f) ? 0.0f : fminf(__frcp_rn(eff), FLT_MAX);
         return (uint32_t)(e + 127);
     } else {
         const float t = __fdiv_rn(amax, denom);
@@ -215,7 +226,7 @@ quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
     int64_t rt, ct;
     locate_tile(b, blockIdx.x, TILE_C, k, rt, ct);
     float gs = 1.0f, denom = 6.0f;
-    if (FMT == kNv) {
+    if (FMT != kMx) {
         gs = __ldg(b.gs[k]);
         denom = __fmul_rn(6.0f, gs);
     }
@@ -387,7 +398,7 @@ quantize_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
     const int64_t nct = rows / TILE_K;
 
     float gs = 1.0f, denom = 6.0f;
-    if (FMT == kNv) {
+    if (FMT != kMx) {
         gs = __ldg(gs_ptr);
         denom = __fmul_rn(6.0f, gs);
     }
@@ -626,6 +637,8 @@ cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, 
         if (tiles > 0x7FFFFFFF) return cudaErrorInvalidValue;
         if (fmt == kNv)
             quantize_rowwise_tiles_kernel<kNv><<<(unsigned)tiles, kThreads, 0, s>>>(b);
+        else if (fmt == kP1)
+            quantize_rowwise_tiles_kernel<kP1><<<(unsigned)tiles, kThreads, 0, s>>>(b);
         else
             quantize_rowwise_tiles_kernel<kMx><<<(unsigned)tiles, kThreads, 0, s>>>(b);
         const cudaError_t e = cudaGetLastError();
@@ -647,6 +660,8 @@ cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, 
         dim3 grid((unsigned)(rows / (4 * kb)), (unsigned)((cols + 127) / 128));
         if (fmt == kNv)
             quantize_colwise_kernel<kNv><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
+        else if (fmt == kP1)
+            quantize_colwise_kernel<kP1><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
         else
             quantize_colwise_kernel<kMx><<<grid, kThreads, 0, s>>>(x, rows, cols, ld, packed, scales, gs);
     }

@@ -11,7 +11,7 @@ import re
 
 import torch
 
-NVFP4, MXFP4 = 0, 1
+NVFP4, MXFP4, P1E8 = 0, 1, 2   # P1E8: 16-element blocks, E8M0 scale under S_global (quantizer only)
 ROWWISE, COLWISE = 0, 1
 GEMM_AUTO, GEMM_PREFILL, GEMM_DECODE = 0, 1, 2
 GEMM_B_STATIC = 0x100   # flag: B / sB not written by a kernel still running on the stream

@@ -56,7 +56,13 @@ typedef enum {
     FP4_NVFP4 = 0,
     /* 32-element blocks, E8M0 power-of-two block scale ([MXFP4-kc],
      * [MXFP4-BW] "32-Element Blocks"). */
-    FP4_MXFP4 = 1
+    FP4_MXFP4 = 1,
+    /* 16-element blocks with an E8M0 block scale under an FP32 S_global:
+     * S_block = 2^ceil(log2(max(amax / (6 S_global), 1e-8))) (capped at
+     * 2^127), the NVFP4 of [NVFP4-Arch] "1. The Dual-Level Mathematical
+     * Formulation" read literally (its block scale is E8M0).  Quantizer only:
+     * the GEMM entry points reject it. */
+    FP4_P1E8 = 2
 } fp4_format;
 
 typedef enum {
@@ -106,8 +112,8 @@ const char* fp4_last_error(void);
 size_t fp4_packed_bytes(int64_t rows, int64_t k);
 
 /* Bytes of the tiled scale buffer for `rows` rows of length k in format
- * `fmt`: ceil(rows/128) * ceil(k/blk/4) * 512 (blk = 16 or 32).  0 for an
- * invalid format. */
+ * `fmt`: ceil(rows/128) * ceil(k/blk/4) * 512 (blk = 16 for NVFP4 and
+ * P1E8, 32 for MXFP4).  0 for an invalid format. */
 size_t fp4_scale_bytes(fp4_format fmt, int64_t rows, int64_t k);
 
 /*
@@ -130,12 +136,14 @@ fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t c
  * q_i = Quantize_E2M1(x_i / (S_global * S_block,j))) and the emulation script
  * in "End-to-End Implementation" (block amax, 1e-8 clamp, ceil(log2(amax/6))).
  *
- * Per block of k elements (k = 16 NVFP4, 32 MXFP4) with amax = max |x_i|:
+ * Per block of k elements (k = 16 NVFP4 and P1E8, 32 MXFP4), amax = max |x_i|:
  *   MXFP4: e = ceil(log2(max(amax, 1e-8) / 6)); scale byte = e + 127;
  *          v_i = x_i * 2^-e.
  *   NVFP4: t = amax / (6 * gs) (FP32); scale byte = E4M3 round-to-nearest-
  *          even of t, saturating at 448; eff = E4M3(byte) * gs (FP32);
  *          v_i = x_i * RN(1/eff) (0 when eff == 0).
+ *   P1E8:  a = max(amax / (6 * gs) (FP32), 1e-8); e = ceil(log2 a), at most
+ *          127; scale byte = e + 127; eff = 2^e * gs (FP32); v_i as NVFP4.
  *   q_i  = E2M1 round-to-nearest-even of v_i, |v| >= 6 -> 6, sign of x_i kept.
  *
  *   axis = FP4_ROWWISE: blocks along each row of in[rows x cols];
@@ -144,8 +152,8 @@ fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t c
  *   axis = FP4_COLWISE: blocks down each column; packed_out is
  *          [cols x rows/2] (the transpose), scales_out covers cols x rows/k.
  *          Requires rows % (4k) == 0 and cols % 8 == 0.
- *   global_scale: device pointer to S_global (NVFP4, required); ignored and
- *          may be NULL for MXFP4.
+ *   global_scale: device pointer to S_global (NVFP4 and P1E8, required);
+ *          ignored and may be NULL for MXFP4.
  *   Sizes of the outputs: fp4_packed_bytes / fp4_scale_bytes with the output
  *   row count and the blocked length.
  */
@@ -169,7 +177,7 @@ typedef struct {
     int64_t rows, cols, ld;
     void* packed_out;           /* device, rows x cols/2 bytes */
     void* scales_out;           /* device, fp4_scale_bytes(fmt, rows, cols) bytes */
-    const float* global_scale;  /* device S_global (NVFP4, required); NULL for MXFP4 */
+    const float* global_scale;  /* device S_global (NVFP4, P1E8: required); NULL for MXFP4 */
 } fp4_quantize_desc;
 
 fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* descs,

@@ -10,7 +10,7 @@ from gpu_util import Guarded, to_dev_bf16, to_dev_f32
 
 pytestmark = pytest.mark.gpu
 
-FMTS = [fp4.NVFP4, fp4.MXFP4]
+FMTS = [fp4.NVFP4, fp4.MXFP4, fp4.P1E8]   # P1E8: 16-element blocks, E8M0 scale under S_global
 
 
 def gpu_quantize(fmt, axis, x_bits, gs):
@@ -19,7 +19,7 @@ def gpu_quantize(fmt, axis, x_bits, gs):
     x = to_dev_bf16(x_bits)
     packed = Guarded(out_rows * K // 2)
     scales = Guarded(fp4.fp4_scale_bytes(fmt, out_rows, K), fill=0x5A)
-    gsd = to_dev_f32(gs) if fmt == fp4.NVFP4 else None
+    gsd = to_dev_f32(gs) if fmt != fp4.MXFP4 else None
     fp4.fp4_quantize(fmt, axis, x, packed.view, scales.view, gsd)
     torch.cuda.synchronize()
     assert fp4.fp4_get_device_status() == 0
@@ -29,7 +29,7 @@ def gpu_quantize(fmt, axis, x_bits, gs):
 
 def check(orc, fmt, axis, x_bits, gs=None):
     if gs is None:
-        gs = orc.global_scale(x_bits) if fmt == fp4.NVFP4 else 1.0
+        gs = orc.global_scale(x_bits) if fmt != fp4.MXFP4 else 1.0
     p_gpu, s_gpu = gpu_quantize(fmt, axis, x_bits, gs)
     p_orc, s_orc = orc.quantize(fmt, axis, x_bits, gs=gs)
     bad = np.argwhere(p_gpu != p_orc)
@@ -87,7 +87,7 @@ def test_rounding_ties_and_extremes(orc, fmt):
         vals[0] = 6.0 * S   # amax = 6 S gives exponent e (MX)
         rows.append(vals)
     x = np.array(rows * 4, dtype=np.float32)
-    x = np.concatenate([x] * (128 // k), axis=1) if fmt == fp4.NVFP4 else np.concatenate([x] * 4, axis=1)
+    x = np.concatenate([x] * (128 // k), axis=1) if k == 16 else np.concatenate([x] * 4, axis=1)
     xb = synth.f32_to_bf16_bits(x)
     extremes = np.array([0x7F7F, 0xFF7F, 0x0001, 0x8001, 0x0080, 0x007F, 0x3F80, 0xBF80],
                         dtype=np.uint16)
@@ -97,11 +97,14 @@ def test_rounding_ties_and_extremes(orc, fmt):
     check(orc, fmt, fp4.ROWWISE, xb)
 
 
-def test_nv_custom_global_scales(orc):
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.P1E8])
+def test_custom_global_scales(orc, fmt):
+    # includes S_global so small that the effective block scale underflows
+    # to zero (all codes +-0) and so large that every ratio is tiny
     x = synth.normal_bf16(256, 512, seed=24, outlier_factor=100.0)
-    for gs in [1.0, 2.0 ** -12, 0.0371, 1000.0]:
-        check(orc, fp4.NVFP4, fp4.ROWWISE, x, gs=gs)
-        check(orc, fp4.NVFP4, fp4.COLWISE, x, gs=gs)
+    for gs in [1.0, 2.0 ** -12, 0.0371, 1000.0, 1e-38, 3e38]:
+        check(orc, fmt, fp4.ROWWISE, x, gs=gs)
+        check(orc, fmt, fp4.COLWISE, x, gs=gs)
 
 
 @pytest.mark.parametrize("shape", [(1, 8), (128, 512), (333, 4104), (4096, 4096)])
@@ -139,9 +142,9 @@ def test_alpha_from_global_scales():
 # --------------------------------------------------------------------------
 def sampled_rows_check(orc, fmt, axis, x_bits, n_rows=48):
     rows, cols = x_bits.shape
-    gs = orc.global_scale(x_bits) if fmt == fp4.NVFP4 else 1.0
+    gs = orc.global_scale(x_bits) if fmt != fp4.MXFP4 else 1.0
     x = to_dev_bf16(x_bits)
-    packed, scales = fp4.quantize(x, fmt, axis, to_dev_f32(gs) if fmt == fp4.NVFP4 else None)
+    packed, scales = fp4.quantize(x, fmt, axis, to_dev_f32(gs) if fmt != fp4.MXFP4 else None)
     torch.cuda.synchronize()
     assert fp4.fp4_get_device_status() == 0
     out_rows, K = (rows, cols) if axis == fp4.ROWWISE else (cols, rows)
@@ -164,12 +167,18 @@ def sampled_rows_check(orc, fmt, axis, x_bits, n_rows=48):
     return gs
 
 
-@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4])
 @pytest.mark.parametrize("axis", [fp4.ROWWISE, fp4.COLWISE])
 @pytest.mark.parametrize("shape", [(16384, 16384), (8192, 28672)])
 def test_full_size_sweep_sampled(orc, fmt, axis, shape):
     x = synth.quant_sweep(*shape)
     sampled_rows_check(orc, fmt, axis, x)
+
+
+@pytest.mark.parametrize("axis", [fp4.ROWWISE, fp4.COLWISE])
+def test_full_size_sweep_sampled_p1e8(orc, axis):
+    x = synth.quant_sweep(16384, 16384)
+    sampled_rows_check(orc, fp4.P1E8, axis, x)
 
 
 @pytest.mark.parametrize("shape", [(1, 8192), (4, 8192), (16, 8192), (16, 512), (3, 64), (1, 64),
@@ -221,11 +230,11 @@ def test_batch_matches_oracle_per_tensor(orc, fmt):
     items, expect = [], []
     for i, (r, c) in enumerate(shapes):
         x = synth.normal_bf16(max(r, 1), c, seed=50 + i, outlier_factor=60.0, zero_frac=0.02)[:r]
-        gs = orc.global_scale(x) if (fmt == fp4.NVFP4 and r > 0) else 1.0
+        gs = orc.global_scale(x) if (fmt != fp4.MXFP4 and r > 0) else 1.0
         packed = Guarded(max(1, r * c // 2))
         scales = Guarded(max(1, fp4.fp4_scale_bytes(fmt, r, c)), fill=0x5A)
         xd = to_dev_bf16(x) if r > 0 else torch.empty((0, c), dtype=torch.bfloat16, device="cuda")
-        items.append((xd, packed.view, scales.view, to_dev_f32(gs) if fmt == fp4.NVFP4 else None))
+        items.append((xd, packed.view, scales.view, to_dev_f32(gs) if fmt != fp4.MXFP4 else None))
         expect.append((x, gs, packed, scales))
     fp4.fp4_quantize_batch(fmt, items)
     torch.cuda.synchronize()
