@@ -372,6 +372,41 @@ class QuantWorkload(Workload):
         return self.qbytes / sec_per_step / 1e9
 
 
+class DequantWorkload(Workload):
+    """Reconstruction of the NVFP4 decode weight W 28672x8192 to BF16 (the
+    input a W4A16 path gives a 16-bit GEMM)."""
+    unit = "GB/s"
+
+    def __init__(self, dev, stream=None, N=28672, K=8192, sets=2):
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.name = "NVFP4 dequantize %dx%d to BF16" % (N, K)
+        W = synth.decode_weight()
+        Wd = _dev_bf16(W, dev)
+        gW = fp4.global_scale(Wd)
+        pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
+        del Wd
+        self.calls, self.bufs = [], []
+        for _ in range(sets):
+            out = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+            self.calls.append([[fp4.BoundCall("fp4_dequantize", fp4.NVFP4, fp4._dptr(pW, "packed"),
+                                              fp4._dptr(sW, "scales"), fp4._dptr(gW, "gs"), N, K,
+                                              fp4._dptr(out, "out"), K, fp4._stream(stream))]])
+            self.bufs.append(out)
+        self.keep = (pW, sW, gW)
+        torch.cuda.empty_cache()
+        self.kernels = ["dequantize"]
+        self.qbytes = N * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, N, K) + N * K * 2
+        self.work = {"dequantize": self.qbytes}
+        self.bound = {"dequantize": "hbm"}
+        self.flops = 0.0
+        self.launches_per_step = 1
+        self.dominant = "dequantize"
+        self.l2_note = "%d output copies of %.0f MB > %d MB L2" % (sets, N * K * 2 / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.qbytes / sec_per_step / 1e9
+
+
 class PrefillWorkload(Workload):
     """NVFP4 prefill: activation S_global + quantize per step, weights
     quantized once, D = A_hat W_hat^T on the persistent tensor-core kernel."""
@@ -422,6 +457,8 @@ def make_workload(name, dev, stream):
         return PrefillWorkload(8192, 28672, 8192, dev, stream=stream)
     if name == "prefill_down":
         return PrefillWorkload(8192, 8192, 28672, dev, stream=stream)
+    if name == "dequant_w_nv":
+        return DequantWorkload(dev, stream=stream)
     if name.startswith("quant_"):
         _, shape, f, ax = name.split("_")
         rows, cols = (16384, 16384) if shape == "16384" else (8192, 28672)
@@ -431,7 +468,7 @@ def make_workload(name, dev, stream):
 
 
 WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
-             "prefill_down"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
+             "prefill_down", "dequant_w_nv"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
                                 for f in ("nv", "mx", "p1e8") for a in ("row", "col")]
 
 

@@ -195,6 +195,28 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
     return FP4_OK;
 }
 
+fp4_status fp4_dequantize(fp4_format fmt, const void* packed, const void* scales,
+                          const float* global_scale, int64_t rows, int64_t k, void* out_bf16,
+                          int64_t ld, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_quant_fmt(fmt) || rows < 0 || k < 0 || ld < k) return FP4_ERR_INVALID_ARG;
+    if (rows == 0 || k == 0) return FP4_OK;
+    if (!packed || !scales || !out_bf16) return FP4_ERR_INVALID_ARG;
+    if (fmt != FP4_MXFP4 && !global_scale) return FP4_ERR_INVALID_ARG;
+    if (k % (4 * fp4::block_size(fmt)) != 0 || rows >= kMaxRows || k >= kMaxRows)
+        return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld % 8 != 0 || !aligned16(packed) || !aligned16(out_bf16)) return FP4_ERR_MISALIGNED;
+    if (global_scale && (reinterpret_cast<uintptr_t>(global_scale) & 3u)) return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_dequantize(
+        (int)fmt, static_cast<const uint8_t*>(packed), static_cast<const uint8_t*>(scales),
+        fmt != FP4_MXFP4 ? global_scale : nullptr, rows, k, static_cast<uint16_t*>(out_bf16), ld,
+        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 fp4_status fp4_quantize_dynamic(fp4_format fmt, const void* in_bf16, int64_t rows, int64_t cols,
                                 int64_t ld, void* packed_out, void* scales_out, float* gs_out,
                                 const float* other_gs, float* alpha_out, fp4_stream_t stream)

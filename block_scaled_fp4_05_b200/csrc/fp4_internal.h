@@ -33,7 +33,9 @@ cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t col
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,
                             int64_t ld, uint8_t* packed, uint8_t* scales, const float* gs,
                             cudaStream_t s);
-// Rowwise quantization of n tensors, batched into persistent launches.
+cudaError_t launch_dequantize(int fmt, const uint8_t* packed, const uint8_t* scales, const float* gs,
+                              int64_t rows, int64_t k, uint16_t* out, int64_t ld, cudaStream_t s);
+// Rowwise quantization of n tensors, batched into one launch per 8.
 struct RowwiseDesc {
     const uint16_t* x;
     int64_t rows, cols, ld;

@@ -18,6 +18,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cstdint>
 #include <cfloat>
 
@@ -232,6 +233,74 @@ quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
     }
     rowwise_tile<FMT>(b.x[k], b.rows[k], b.cols[k], b.ld[k], b.packed[k], b.scales[k], rt, ct, gs, denom,
                       s_tile);
+}
+
+// ---------------------------------------------------------------------------
+// Dequantization (reconstruction) x_hat = q * S_block (* S_global) of a
+// rowwise-quantized operand [rows x k] into BF16, rounded once to nearest
+// even: the product of the E2M1 value, the block scale and S_global is exact
+// in FP64 (at most 2 + 4 + 24 significant bits), then converted.  Thread t
+// takes 16 packed bytes (32 codes) of one row; HBM-bound (0.5 + 1/blk bytes
+// read, 2 written per element).
+// ---------------------------------------------------------------------------
+template <int FMT>
+__global__ void __launch_bounds__(kThreads)
+dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
+                  const float* __restrict__ gs_ptr, int64_t rows, int64_t k, uint16_t* __restrict__ out,
+                  int64_t ld)
+{
+    pdl_trigger();
+    constexpr int KB = FMT == kMx ? 32 : 16;
+    const double gs = FMT != kMx ? (double)__ldg(gs_ptr) : 1.0;
+    const int64_t cpr = k / 32;                         // 16-byte packed chunks per row
+    const int64_t nsc = k / KB;                         // scales per row
+    const int64_t nct = (nsc + 3) / 4;                  // scale tiles per 128-row group
+    const int64_t total = rows * cpr;
+    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total;
+         u += (int64_t)gridDim.x * kThreads) {
+        const int64_t r = u / cpr, c = u - r * cpr;
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(packed + r * (k / 2)) + c);
+        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+        uint32_t o[16];
+#pragma unroll
+        for (int b = 0; b < 32 / KB; ++b) {
+            const int64_t blk = c * (32 / KB) + b;      // block index within the row
+            const uint8_t sb = __ldg(scales + ((r / 128) * nct + blk / 4) * 512 + (r % 32) * 16 +
+                                     ((r / 32) % 4) * 4 + blk % 4);
+            double s;
+            if (FMT == kNv) {
+                s = (double)e4m3_value(sb);
+            } else {
+                s = __longlong_as_double((long long)(sb + 896) << 52);   // 2^(sb - 127), exact
+            }
+            const double eff = s * gs;
+            // BF16 of the 8 magnitudes q * eff (q = 0, .5, 1, 1.5, 2, 3, 4, 6),
+            // each exact in FP64 and rounded once; the sign of a code is the
+            // BF16 sign bit (rounding to nearest even is symmetric)
+            constexpr double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+            uint32_t t[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                t[j] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(kE2M1[2 * j] * eff)) |
+                       ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(kE2M1[2 * j + 1] * eff)) << 16);
+            auto lookup = [&](uint32_t nib) {
+                const uint32_t lo = (nib & 2u) ? t[1] : t[0];
+                const uint32_t hi = (nib & 2u) ? t[3] : t[2];
+                const uint32_t w2 = (nib & 4u) ? hi : lo;
+                const uint32_t mag = (nib & 1u) ? (w2 >> 16) : (w2 & 0xFFFFu);
+                return mag | ((nib & 8u) << 12);
+            };
+#pragma unroll
+            for (int i = 0; i < KB / 2; ++i) {          // two codes per output word
+                const int e = b * KB + 2 * i;           // element within the 32
+                const uint32_t byte = (words[e / 8] >> ((e % 8) * 4)) & 0xFFu;
+                o[e / 2] = lookup(byte & 0xFu) | (lookup(byte >> 4) << 16);
+            }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(out + r * ld + c * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -645,6 +714,26 @@ cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, 
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+cudaError_t launch_dequantize(int fmt, const uint8_t* packed, const uint8_t* scales, const float* gs,
+                              int64_t rows, int64_t k, uint16_t* out, int64_t ld, cudaStream_t s)
+{
+    if (rows == 0 || k == 0) return cudaSuccess;
+    DeviceInfo dev;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess) return e;
+    const int64_t chunks = rows * (k / 32);
+    int64_t grid = (chunks + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)dev.sm_count * 8;
+    if (grid > cap) grid = cap;
+    if (fmt == kNv)
+        dequantize_kernel<kNv><<<(unsigned)grid, kThreads, 0, s>>>(packed, scales, gs, rows, k, out, ld);
+    else if (fmt == kP1)
+        dequantize_kernel<kP1><<<(unsigned)grid, kThreads, 0, s>>>(packed, scales, gs, rows, k, out, ld);
+    else
+        dequantize_kernel<kMx><<<(unsigned)grid, kThreads, 0, s>>>(packed, scales, gs, rows, k, out, ld);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_quantize(int fmt, int axis, const uint16_t* x, int64_t rows, int64_t cols,

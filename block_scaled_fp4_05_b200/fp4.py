@@ -62,6 +62,8 @@ def lib():
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
+        L.fp4_dequantize.restype = c.c_int
+        L.fp4_dequantize.argtypes = [c.c_int, P, P, P, i64, i64, P, i64, st]
         L.fp4_quantize_batch.restype = c.c_int
         L.fp4_quantize_batch.argtypes = [c.c_int, c.c_int, P, st]
         L.fp4_quantize_dynamic.restype = c.c_int
@@ -150,6 +152,15 @@ def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream
                               _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
                               _dptr(global_scale, "global_scale"), _stream(stream)),
            "fp4_quantize")
+
+
+def fp4_dequantize(fmt, packed, scales, global_scale, out, stream=None):
+    """out[rows x k] (bf16) = q * S_block (* S_global), rounded once to BF16."""
+    rows, k = out.shape[0], packed.shape[1] * 2
+    _check(lib().fp4_dequantize(int(fmt), _dptr(packed, "packed"), _dptr(scales, "scales"),
+                                _dptr(global_scale, "global_scale"), rows, k, _dptr(out, "out"),
+                                out.stride(0), _stream(stream)), "fp4_dequantize")
+    return out
 
 
 class QuantizeDesc(ctypes.Structure):

@@ -162,6 +162,24 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
                         const float* global_scale, fp4_stream_t stream);
 
 /*
+ * Reconstruction of a rowwise-quantized operand in BF16:
+ *   out[r, i] = BF16_RNE(q[r, i] * S_block(r, i / k) * S_global)
+ * ([NVFP4-Arch] "1. The Dual-Level Mathematical Formulation",
+ * reconstruction x_hat), with S_global = 1 for MXFP4.  The product is exact
+ * before the single rounding.  This is what a W4A16 path feeds a 16-bit GEMM;
+ * the library's own GEMM never widens its operands.
+ *   packed : device, [rows x k/2] (fp4_quantize's rowwise output)
+ *   scales : device, its scale tiles
+ *   global_scale : device S_global (NVFP4, P1E8: required; MXFP4: ignored)
+ *   out_bf16 : device, [rows x k] BF16 with leading dimension ld (elements)
+ * Requires k % (4 * block size) == 0, ld >= k, ld % 8 == 0, 16-byte aligned
+ * packed and out_bf16.
+ */
+fp4_status fp4_dequantize(fp4_format fmt, const void* packed, const void* scales,
+                          const float* global_scale, int64_t rows, int64_t k, void* out_bf16,
+                          int64_t ld, fp4_stream_t stream);
+
+/*
  * Rowwise quantization of several tensors in one launch (e.g. both GEMM
  * operands of a step), each exactly as fp4_quantize(fmt, FP4_ROWWISE, ...)
  * with its own sizes, buffers and S_global.  One launch covers the 128-row
