@@ -372,6 +372,62 @@ class QuantWorkload(Workload):
         return self.qbytes / sec_per_step / 1e9
 
 
+class MoeWorkload(Workload):
+    """MXFP4 mixture-of-experts up-projection: 8 experts with weights
+    14336 x 4096 and uneven token counts (8192 routed tokens in all), per
+    step the quantization of every expert's activations (one batched launch)
+    and the 8 GEMMs, either as one grouped launch or as 8 separate ones."""
+    TOKENS = [1536, 512, 2048, 768, 1024, 256, 1280, 768]
+
+    def __init__(self, dev, grouped=True, stream=None, N=14336, K=4096, sets=2):
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        fmt = fp4.MXFP4
+        self.name = "MXFP4 MoE up-projection, 8 experts %dx%d, tokens %s, %s" % (
+            N, K, "/".join(str(t) for t in self.TOKENS), "grouped GEMM" if grouped else "8 separate GEMMs")
+        experts = []
+        for e in range(len(self.TOKENS)):
+            W = synth.normal_bf16(N, K, seed=6, tensor_id=100 + e, sigma=0.02)
+            Wd = _dev_bf16(W, dev)
+            experts.append(fp4.quantize(Wd, fmt, fp4.ROWWISE, None))
+            del Wd
+        M_all = sum(self.TOKENS)
+        A = synth.normal_bf16(M_all, K, seed=6, outlier_factor=50.0)
+        self.calls, self.bufs = [], []
+        for _ in range(sets):
+            Ad = _dev_bf16(A, dev)
+            q_items, g_items, views = [], [], []
+            r0 = 0
+            for e, m in enumerate(self.TOKENS):
+                pA, sA = _qbufs(fmt, m, K, dev)
+                D = torch.empty((m, N), dtype=torch.bfloat16, device=dev)
+                q_items.append((Ad[r0:r0 + m], pA, sA, None))
+                g_items.append((pA, sA, experts[e][0], experts[e][1], K, None, D))
+                views.append((pA, sA, D))
+                r0 += m
+            quant = [fp4.bind_quantize_batch(fmt, q_items, stream)]
+            if grouped:
+                gemm = [fp4.bind_gemm_grouped(fmt, g_items, stream)]
+            else:
+                gemm = [fp4.bind_gemm(fmt, it[0], it[1], it[2], it[3], it[6].shape[0], N, K, None, it[6], None,
+                                      fp4.GEMM_PREFILL, stream) for it in g_items]
+            self.calls.append([quant, gemm])
+            self.bufs.append((Ad, views))
+        self.experts = experts
+        torch.cuda.empty_cache()
+        self.kernels = ["quantize", "gemm"]
+        qbytes = M_all * K * 2 + M_all * K // 2 + sum(fp4.fp4_scale_bytes(fmt, m, K) for m in self.TOKENS)
+        self.flops = 2.0 * M_all * N * K
+        self.work = {"quantize": qbytes, "gemm": self.flops}
+        self.bound = {"quantize": "hbm", "gemm": "tensor"}
+        self.launches_per_step = 2 if grouped else 1 + len(self.TOKENS)
+        self.dominant = "gemm"
+        self.l2_note = "expert weights %.0f MB > %d MB L2" % (
+            len(self.TOKENS) * (N * K // 2 + fp4.fp4_scale_bytes(fmt, N, K)) / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.flops / sec_per_step / 1e12
+
+
 class DequantWorkload(Workload):
     """Reconstruction of the NVFP4 decode weight W 28672x8192 to BF16 (the
     input a W4A16 path gives a 16-bit GEMM)."""
@@ -457,6 +513,8 @@ def make_workload(name, dev, stream):
         return PrefillWorkload(8192, 28672, 8192, dev, stream=stream)
     if name == "prefill_down":
         return PrefillWorkload(8192, 8192, 28672, dev, stream=stream)
+    if name in ("moe_grouped_mx", "moe_separate_mx"):
+        return MoeWorkload(dev, grouped=name == "moe_grouped_mx", stream=stream)
     if name == "dequant_w_nv":
         return DequantWorkload(dev, stream=stream)
     if name.startswith("quant_"):
@@ -468,7 +526,7 @@ def make_workload(name, dev, stream):
 
 
 WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
-             "prefill_down", "dequant_w_nv"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
+             "prefill_down", "moe_grouped_mx", "moe_separate_mx", "dequant_w_nv"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
                                 for f in ("nv", "mx", "p1e8") for a in ("row", "col")]
 
 

@@ -6,6 +6,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <vector>
+
 #include "fp4_internal.h"
 
 namespace fp4 {
@@ -264,6 +266,76 @@ size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K)
     return fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
 }
 
+// Checks of one GEMM problem with M, N > 0 (shared by fp4_gemm and
+// fp4_gemm_grouped).
+static fp4_status validate_gemm(fp4_format fmt, const void* A, const void* sA, const void* B,
+                                const void* sB, int64_t M, int64_t N, int64_t K, const float* alpha,
+                                const void* D, int64_t ldd)
+{
+    if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
+    if (!D) return FP4_ERR_INVALID_ARG;
+    const int kq = fmt == FP4_NVFP4 ? 64 : 128;
+    if (K % kq != 0 || N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (M >= kMaxRows || N >= kMaxRows || K / 2 >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldd % 8 != 0 || !aligned16(D)) return FP4_ERR_MISALIGNED;
+    if (K > 0) {
+        if (!A || !sA || !B || !sB) return FP4_ERR_INVALID_ARG;
+        if (!aligned16(A) || !aligned16(B) || !aligned16(sA) || !aligned16(sB))
+            return FP4_ERR_MISALIGNED;
+    }
+    if (alpha && (reinterpret_cast<uintptr_t>(alpha) & 3u)) return FP4_ERR_MISALIGNED;
+    return FP4_OK;
+}
+
+fp4_status fp4_gemm_grouped(fp4_format fmt, int n, const fp4_gemm_problem* problems, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (!valid_fmt(fmt) || n < 0 || (n > 0 && !problems)) return FP4_ERR_INVALID_ARG;
+    int work = 0;
+    for (int i = 0; i < n; ++i) {
+        const fp4_gemm_problem& q = problems[i];
+        if (q.M < 0 || q.N < 0 || q.K < 0) return FP4_ERR_INVALID_ARG;
+        if (q.M == 0 || q.N == 0) continue;
+        const fp4_status vs = validate_gemm(fmt, q.A, q.sA, q.B, q.sB, q.M, q.N, q.K, q.alpha, q.D, q.ldd);
+        if (vs != FP4_OK) return vs;
+        ++work;
+    }
+    if (work == 0) return FP4_OK;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    if (!fp4::tensor_map_encoder_available()) return FP4_ERR_NO_DEVICE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<fp4::GemmArgs> args;
+    args.reserve(n);
+    for (int i = 0; i < n; ++i) {
+        const fp4_gemm_problem& q = problems[i];
+        if (q.M == 0 || q.N == 0) continue;
+        if (q.K == 0) {   // D = 0
+            st = from_cuda(cudaMemset2DAsync(q.D, (size_t)q.ldd * 2, 0, (size_t)q.N * 2, (size_t)q.M, s));
+            if (st != FP4_OK) return st;
+            continue;
+        }
+        fp4::GemmArgs a;
+        a.fmt = (int)fmt;
+        a.A = static_cast<const uint8_t*>(q.A);
+        a.sA = static_cast<const uint8_t*>(q.sA);
+        a.B = static_cast<const uint8_t*>(q.B);
+        a.sB = static_cast<const uint8_t*>(q.sB);
+        a.M = q.M;
+        a.N = q.N;
+        a.K = q.K;
+        a.alpha = q.alpha;
+        a.D = static_cast<uint16_t*>(q.D);
+        a.ldd = q.ldd;
+        a.ws = nullptr;
+        a.ws_bytes = 0;
+        a.b_static = false;
+        args.push_back(a);
+    }
+    return from_cuda(fp4::launch_gemm_grouped((int)args.size(), args.data(), dev, s));
+}
+
 fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, const void* B,
                                 const void* sB, int64_t M, int64_t N, int64_t K,
                                 const float* alpha, void* D, int64_t ldd, void* workspace,
@@ -276,19 +348,12 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
     if (kernel != FP4_GEMM_AUTO && kernel != FP4_GEMM_PREFILL && kernel != FP4_GEMM_DECODE)
         return FP4_ERR_INVALID_ARG;
     if (flags & ~(int)FP4_GEMM_B_STATIC) return FP4_ERR_INVALID_ARG;
-    if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
-    if (M == 0 || N == 0) return FP4_OK;
-    if (!D) return FP4_ERR_INVALID_ARG;
-    const int kq = fmt == FP4_NVFP4 ? 64 : 128;
-    if (K % kq != 0 || N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (M >= kMaxRows || N >= kMaxRows || K / 2 >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
-    if (ldd % 8 != 0 || !aligned16(D)) return FP4_ERR_MISALIGNED;
-    if (K > 0) {
-        if (!A || !sA || !B || !sB) return FP4_ERR_INVALID_ARG;
-        if (!aligned16(A) || !aligned16(B) || !aligned16(sA) || !aligned16(sB))
-            return FP4_ERR_MISALIGNED;
+    if (M == 0 || N == 0) {
+        if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
+        return FP4_OK;
     }
-    if (alpha && (reinterpret_cast<uintptr_t>(alpha) & 3u)) return FP4_ERR_MISALIGNED;
+    const fp4_status vs = validate_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, ldd);
+    if (vs != FP4_OK) return vs;
     fp4::DeviceInfo dev;
     fp4_status st = require_device(&dev);
     if (st != FP4_OK) return st;

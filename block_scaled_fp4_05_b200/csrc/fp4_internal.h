@@ -63,6 +63,7 @@ struct GemmArgs {
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);
+cudaError_t launch_gemm_grouped(int n, const GemmArgs* a, const DeviceInfo& dev, cudaStream_t s);
 cudaError_t read_and_clear_error_word(unsigned int* word);
 cudaError_t launch_wait_selftest(cudaStream_t s);
 size_t noalloc_scratch_bytes();

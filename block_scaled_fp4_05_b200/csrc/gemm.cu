@@ -1050,10 +1050,23 @@ __device__ __forceinline__ void spin_ns(uint64_t ns)
     }
 }
 
-template <int STAGES, bool MX>
+// The problems one pair-kernel launch computes: NG = 1 for fp4_gemm, up to
+// kMaxGroups for fp4_gemm_grouped.  Tile t of the launch belongs to problem g
+// with tile_begin[g] <= t < tile_begin[g + 1]; within a problem, M tiles
+// run fastest.
+constexpr int kMaxGroups = 16;
+
+template <int NG>
+struct PairArgs {
+    CUtensorMap a[NG], b[NG], d[NG];   // A, B (K-major, 128-byte swizzle) and D of each problem
+    Params p[NG];
+    int n;
+    int tile_begin[NG + 1];
+};
+
+template <int STAGES, bool MX, int NG>
 __global__ void __launch_bounds__(kThreads, 1)
-fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmD, const Params p)
+fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
 {
     using C = PairCfg<STAGES, MX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1107,20 +1120,32 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
-    const int tiles = p.tiles_m * p.tiles_n;
+    const int tiles = args.tile_begin[args.n];
+    // problem and its local tile index of launch tile t
+    auto locate = [&](int t, int& g, int& lt) {
+        g = 0;
+        if (NG > 1)
+            while (g + 1 < args.n && t >= args.tile_begin[g + 1]) ++g;
+        lt = t - args.tile_begin[g];
+    };
 
     if (warp == 0) {
         // ---------------- TMA producer (both CTAs) ----------------
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-            const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
+            for (int g = 0; g < args.n; ++g) {
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&args.a[g])) : "memory");
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&args.b[g])) : "memory");
+            }
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
             pdl_wait();
             for (int t = pair; ok && t < tiles; t += npairs) {
-                const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+                int g, lt;
+                locate(t, g, lt);
+                const Params& p = args.p[g];
+                const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
+                const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
                 const int rta = tm * 2 + (int)rank;                // this CTA's 128-row A tile
                 const bool has_sfa = rta < p.sfa_row_tiles;
                 int nbh = 0;
@@ -1143,8 +1168,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     if (leader)
                         mbar_arrive_expect_tx(B_FULL(stage), 2u * (A_BYTES + C::B_BYTES));
                     const uint32_t full_leader = map_to_rank(B_FULL(stage), 0);
-                    tma_load_2d_pair(&tmA, full_leader, st, ks * BK_BYTES, ya);
-                    tma_load_2d_pair(&tmB, full_leader, st + C::OFF_B, ks * BK_BYTES, yb);
+                    tma_load_2d_pair(&args.a[g], full_leader, st, ks * BK_BYTES, ya);
+                    tma_load_2d_pair(&args.b[g], full_leader, st + C::OFF_B, ks * BK_BYTES, yb);
                     mbar_arrive_expect_tx(B_SFFULL(stage), sf_bytes * ((has_sfa ? 1 : 0) + nbh));
                     if (has_sfa)
                         bulk_load(st + C::OFF_SFA, sfa_row + ct0 * SF_CHUNK, sf_bytes, B_SFFULL(stage));
@@ -1177,6 +1202,9 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int t = pair; ok && t < tiles; t += npairs) {
+                int g, lt;
+                locate(t, g, lt);
+                const Params& p = args.p[g];
                 if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
                 tc_fence_after();
                 for (int ks = 0; ks < p.ks_total; ++ks) {
@@ -1229,11 +1257,14 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         const int q = warp & 3;
         const int row = q * 32 + lane;
         pdl_wait();
-        const float alpha = p.alpha ? *p.alpha : 1.0f;
         const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
         const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
         for (int t = pair; t < tiles; t += npairs) {
+            int g, lt;
+            locate(t, g, lt);
+            const Params& p = args.p[g];
+            const float alpha = p.alpha ? *p.alpha : 1.0f;
             int ok = 0;
             if (lane == 0) ok = wait_bounded(acc_full, acc_phase, abort_flag, ERR_ACC_FULL) ? 1 : 0;
             ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -1263,7 +1294,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             // time go to its staging block (64-byte rows; 16-byte chunk j of
             // row r at chunk j ^ ((r >> 1) & 3), the 64-byte swizzle), then
             // one lane stores the block with TMA, coalesced and clipped to D.
-            const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+            const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
             const int y0 = (tm * 2 + (int)rank) * BM + q * 32;
             const uint32_t blk = smem0 + C::OFF_EPI + q * C::EPI_BLOCK;
             const uint32_t my_row = blk + lane * 64;
@@ -1283,7 +1314,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                                      : "memory");
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&tmD, blk, x0, y0);
+                    if (lane == 0) tma_store_2d(&args.d[g], blk, x0, y0);
                 }
             }
             acc_phase ^= 1u;
@@ -1296,7 +1327,10 @@ fp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint32_t phase = 0;
         bool ok = true;
         for (int t = pair; ok && t < tiles; t += npairs) {
-            const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+            int g, lt;
+            locate(t, g, lt);
+            const Params& p = args.p[g];
+            const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
             const bool has_sfa = tm * 2 + (int)rank < p.sfa_row_tiles;
             int nbh = 0;
             for (int h = 0; h < 2; ++h)
@@ -1575,12 +1609,11 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.max_seg = 0;
 }
 
-template <int STAGES, bool MX>
-cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& td,
-                               const Params& p, int grid, cudaStream_t s)
+template <int STAGES, bool MX, int NG>
+cudaError_t launch_pair_kernel(const PairArgs<NG>& args, int grid, cudaStream_t s)
 {
     using C = PairCfg<STAGES, MX>;
-    auto kern = fp4_gemm_pair_kernel<STAGES, MX>;
+    auto kern = fp4_gemm_pair_kernel<STAGES, MX, NG>;
     static std::mutex mu;
     static uint64_t done_mask = 0;
     int dev = 0;
@@ -1611,7 +1644,7 @@ cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, con
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, kern, ta, tb, td, p);
+    e = cudaLaunchKernelEx(&cfg, kern, args);
     if (e != cudaSuccess) set_last_error("pair GEMM kernel launch", e);
     return e;
 }
@@ -1619,23 +1652,65 @@ cudaError_t launch_pair_kernel(const CUtensorMap& ta, const CUtensorMap& tb, con
 constexpr int PAIR_STAGES_NV = 5;   // 38 KB per stage
 constexpr int PAIR_STAGES_MX = 6;   // 35 KB per stage
 
-cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
+// Fills problem slot g of a pair-kernel launch (tensor maps and Params).
+template <int NG>
+bool fill_pair_problem(PairArgs<NG>& args, int g, const GemmArgs& a)
 {
-    CUtensorMap ta, tb, td;
-    if (!make_map(&ta, a.A, a.M, a.K / 2, BM) || !make_map(&tb, a.B, a.N, a.K / 2, PAIR_BHALF) ||
-        !make_map_d(&td, a.D, a.M, a.N, a.ldd)) {
-        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
-        return cudaErrorInvalidValue;
-    }
-    Params p;
+    if (!make_map(&args.a[g], a.A, a.M, a.K / 2, BM) || !make_map(&args.b[g], a.B, a.N, a.K / 2, PAIR_BHALF) ||
+        !make_map_d(&args.d[g], a.D, a.M, a.N, a.ldd))
+        return false;
+    Params& p = args.p[g];
     fill_common(p, a, a.M, a.N, a.sA, a.sB);
     p.tiles_m = (int32_t)((a.M + 255) / 256);
     p.tiles_n = (int32_t)((a.N + PAIR_BN - 1) / PAIR_BN);
-    const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
+    args.tile_begin[g + 1] = args.tile_begin[g] + p.tiles_m * p.tiles_n;
+    return true;
+}
+
+template <int NG>
+cudaError_t launch_pair(const PairArgs<NG>& args, int fmt, const DeviceInfo& dev, cudaStream_t s)
+{
+    const int64_t tiles = args.tile_begin[args.n];
+    if (tiles == 0) return cudaSuccess;
     const int64_t max_pairs = dev.sm_count / 2;
     const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
-    if (a.fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true>(ta, tb, td, p, grid, s);
-    return launch_pair_kernel<PAIR_STAGES_NV, false>(ta, tb, td, p, grid, s);
+    if (fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true, NG>(args, grid, s);
+    return launch_pair_kernel<PAIR_STAGES_NV, false, NG>(args, grid, s);
+}
+
+cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
+{
+    PairArgs<1> args;
+    args.n = 1;
+    args.tile_begin[0] = 0;
+    if (!fill_pair_problem(args, 0, a)) {
+        set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+        return cudaErrorInvalidValue;
+    }
+    return launch_pair(args, a.fmt, dev, s);
+}
+
+// Several problems per launch, kMaxGroups at a time; problems with M == 0 or
+// N == 0 are skipped, K == 0 is handled by the caller.
+cudaError_t launch_gemm_grouped(int n, const GemmArgs* a, const DeviceInfo& dev, cudaStream_t s)
+{
+    for (int i0 = 0; i0 < n; i0 += kMaxGroups) {
+        PairArgs<kMaxGroups> args;
+        args.n = 0;
+        args.tile_begin[0] = 0;
+        for (int i = i0; i < n && i < i0 + kMaxGroups; ++i) {
+            if (a[i].M == 0 || a[i].N == 0 || a[i].K == 0) continue;
+            if (!fill_pair_problem(args, args.n, a[i])) {
+                set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
+                return cudaErrorInvalidValue;
+            }
+            ++args.n;
+        }
+        if (args.n == 0) continue;
+        const cudaError_t e = launch_pair(args, a[i0].fmt, dev, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)

@@ -62,6 +62,8 @@ def lib():
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
+        L.fp4_gemm_grouped.restype = c.c_int
+        L.fp4_gemm_grouped.argtypes = [c.c_int, c.c_int, P, st]
         L.fp4_dequantize.restype = c.c_int
         L.fp4_dequantize.argtypes = [c.c_int, P, P, P, i64, i64, P, i64, st]
         L.fp4_quantize_batch.restype = c.c_int
@@ -152,6 +154,39 @@ def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream
                               _dptr(packed_out, "packed_out"), _dptr(scales_out, "scales_out"),
                               _dptr(global_scale, "global_scale"), _stream(stream)),
            "fp4_quantize")
+
+
+class GemmProblem(ctypes.Structure):
+    """fp4_gemm_problem of include/fp4.h."""
+    _fields_ = [("A", ctypes.c_void_p), ("sA", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("sB", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("alpha", ctypes.c_void_p), ("D", ctypes.c_void_p),
+                ("ldd", ctypes.c_int64)]
+
+
+def _gemm_problems(items):
+    arr = (GemmProblem * max(1, len(items)))()
+    for i, (A, sA, B, sB, K, alpha, D) in enumerate(items):
+        arr[i] = GemmProblem(_dptr(A, "A"), _dptr(sA, "sA"), _dptr(B, "B"), _dptr(sB, "sB"),
+                             D.shape[0], D.shape[1], int(K), _dptr(alpha, "alpha"), _dptr(D, "D"),
+                             D.stride(0))
+    return arr
+
+
+def fp4_gemm_grouped(fmt, items, stream=None):
+    """Grouped GEMM; items are (A, sA, B, sB, K, alpha or None, D) tuples with
+    D [M x N] bf16 (M, N taken from D)."""
+    arr = _gemm_problems(items)
+    _check(lib().fp4_gemm_grouped(int(fmt), len(items), ctypes.cast(arr, ctypes.c_void_p), _stream(stream)),
+           "fp4_gemm_grouped")
+
+
+def bind_gemm_grouped(fmt, items, stream=None):
+    arr = _gemm_problems(items)
+    call = BoundCall("fp4_gemm_grouped", int(fmt), len(items), ctypes.cast(arr, ctypes.c_void_p),
+                     _stream(stream))
+    call.keep = arr
+    return call
 
 
 def fp4_dequantize(fmt, packed, scales, global_scale, out, stream=None):

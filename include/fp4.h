@@ -271,6 +271,31 @@ fp4_status fp4_gemm_with_kernel(fp4_format fmt, const void* A, const void* sA, c
                                 const float* alpha, void* D, int64_t ldd, void* workspace,
                                 size_t ws_bytes, fp4_gemm_kernel kernel, fp4_stream_t stream);
 
+/*
+ * Grouped GEMM: n independent problems D_i = alpha_i * A_i_hat * B_i_hat^T
+ * (e.g. the experts of a mixture-of-experts layer, each with its own token
+ * count M_i), each with the semantics and requirements of fp4_gemm, computed
+ * by one persistent launch of the prefill kernel per 16 problems: the
+ * 256 x 256 tiles of all problems form one list over the CTA pairs, so small
+ * problems share the GPU instead of each paying a launch and a partial
+ * wave.  Problems with M_i == 0 or N_i == 0 are skipped; K_i == 0 writes
+ * zeros.  Every problem is validated before anything is launched.
+ *   problems : host array of n descriptors (the pointers in them are device)
+ */
+typedef struct {
+    const void* A;       /* packed [M x K/2] */
+    const void* sA;      /* its scales */
+    const void* B;       /* packed [N x K/2] */
+    const void* sB;      /* its scales */
+    int64_t M, N, K;
+    const float* alpha;  /* device, or NULL for 1.0 */
+    void* D;             /* BF16 [M x N], leading dimension ldd */
+    int64_t ldd;
+} fp4_gemm_problem;
+
+fp4_status fp4_gemm_grouped(fp4_format fmt, int n, const fp4_gemm_problem* problems,
+                            fp4_stream_t stream);
+
 /* Workspace bytes the decode kernel needs for this shape on the current
  * device: 64 KB of counters plus the split-K partials (0 when the decode
  * kernel does not apply, i.e. M > 16 or N > 524288). */

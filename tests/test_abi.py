@@ -111,3 +111,25 @@ def test_p1e8_is_a_quantizer_format_only(orc):
     g = L.fp4_gemm_with_kernel
     assert g(2, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 1
     assert L.fp4_gemm_workspace_bytes(2, 16, 1024, 1024) == 0
+
+
+def test_gemm_grouped_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    G = fp4.GemmProblem
+
+    def call(fmt, probs):
+        arr = (G * max(1, len(probs)))(*probs)
+        return L.fp4_gemm_grouped(fmt, len(probs), ctypes.cast(arr, P), None)
+
+    a = 1 << 20
+    good = G(a, a, a, a, 16, 16, 64, None, a, 16)
+    assert call(9, [good]) == 1                                         # bad format
+    assert call(2, [good]) == 1                                         # P1E8: quantizer only
+    assert L.fp4_gemm_grouped(0, -1, None, None) == 1
+    assert call(0, [good, G(a, a, a, a, 16, 16, 96, None, a, 16)]) == 2  # K % 64
+    assert call(0, [good, G(a, a, a, a, 16, 12, 64, None, a, 16)]) == 2  # N % 8
+    assert call(0, [G(a + 1, a, a, a, 16, 16, 64, None, a, 16)]) == 3    # misaligned A
+    assert call(0, [G(0, 0, 0, 0, 0, 16, 64, None, 0, 16)]) == 0         # empty only: no-op
+    if not torch.cuda.is_available():
+        assert call(0, [good]) == 6

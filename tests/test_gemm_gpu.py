@@ -262,3 +262,42 @@ def test_prefill_config_sampled(orc, shape):
     M, N, K = shape
     A, W = synth.prefill(M, N, K)
     sampled_check(orc, fp4.NVFP4, A, W, fp4.GEMM_PREFILL, n_pairs=1024)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_grouped_gemm_matches_oracle_per_problem(orc, fmt):
+    # experts of an MoE layer: one weight shape, token counts from 0 to a few
+    # hundred, plus one problem of another shape and one with K = 0; 18
+    # problems, so the call makes two launches (16 + 2)
+    rng = np.random.default_rng(36)
+    K, N = 1024, 512
+    shapes = [(int(m), N, K) for m in rng.integers(0, 300, 15)] + [(0, N, K), (40, 264, 640), (5, 136, 0)]
+    items, checks = [], []
+    for i, (M, Ni, Ki) in enumerate(shapes):
+        if Ki and Ki % (64 if fmt == fp4.NVFP4 else 128):
+            Ki = 768
+        Ms = max(M, 1)
+        A = synth.normal_bf16(Ms, max(Ki, 128), seed=37 + i, outlier_factor=50.0)[:M, :Ki]
+        W = synth.normal_bf16(Ni, max(Ki, 128), seed=37 + i, tensor_id=1, sigma=0.02)[:, :Ki]
+        D = torch.full((M, Ni + 8), float("nan"), dtype=torch.bfloat16, device="cuda")
+        if M > 0 and Ki > 0:
+            pA, sA, pW, sW, alpha = oracle_operands(orc, fmt, np.ascontiguousarray(A), np.ascontiguousarray(W))
+            items.append((to_dev_u8(pA), to_dev_u8(sA), to_dev_u8(pW), to_dev_u8(sW), Ki, to_dev_f32(alpha),
+                          D[:, :Ni]))
+            checks.append((D, Ni, orc.gemm(fmt, pA, sA, pW, sW, alpha=alpha)))
+        else:
+            z = torch.zeros((64,), dtype=torch.uint8, device="cuda")
+            items.append((z, z, z, z, Ki, None, D[:, :Ni]))
+            checks.append((D, Ni, None))
+    fp4.fp4_gemm_grouped(fmt, items)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    for (M, Ni, Ki), (D, n_cols, want) in zip(shapes, checks):
+        assert torch.isnan(D[:, n_cols:].float()).all()
+        if M == 0:
+            continue
+        if want is None:   # K == 0
+            assert torch.all(D[:, :n_cols].float() == 0)
+            continue
+        D_orc, S = want
+        assert_gemm_close(bf16_dev_to_f64(D[:, :n_cols]), D_orc, S, "grouped %s" % ((M, Ni, Ki),))
