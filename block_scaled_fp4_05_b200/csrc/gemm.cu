@@ -8,7 +8,10 @@
 // in FP32) and "How Microscaling FP4 (MXFP4) Halves Memory Bandwidth...",
 // "Silicon Execution" (accumulate in 32-bit precision before storing).
 //
-// Kernel structure (one CTA per SM, persistent):
+// Two kernels: fp4_gemm_pair_kernel (prefill and grouped problems, CTA pairs,
+// described before its definition) and fp4_gemm_kernel (one CTA per tile,
+// used in the decode form).  Structure of the latter, which the pair kernel
+// shares role for role (one CTA per SM, persistent):
 //   warp 0      TMA producer: packed A/B tiles via tensor maps (128-byte
 //               swizzle), scale chunks via 1-D bulk copies, into a ring of
 //               STAGES shared-memory stages guarded by full/empty mbarriers.
