@@ -73,6 +73,9 @@ fp4_status require_device(fp4::DeviceInfo* dev)
 
 constexpr int64_t kMaxGridY = 65535;
 constexpr int64_t kMaxRows = (int64_t)1 << 31;
+// Rowwise tiles (128 rows x 4 blocks) of one tensor: a batched launch puts
+// the tiles of up to 8 tensors in one 1-D grid.
+constexpr int64_t kMaxRowTiles = (int64_t)1 << 28;
 
 }  // namespace
 
@@ -140,7 +143,8 @@ fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int6
     const int kb = fp4::block_size(fmt);
     if (axis == FP4_ROWWISE) {
         if (cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-        if ((rows + 127) / 128 > kMaxGridY) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (rows >= kMaxRows || cols >= kMaxRows || ((rows + 127) / 128) * (cols / (4 * kb)) > kMaxRowTiles)
+            return FP4_ERR_UNSUPPORTED_SHAPE;
     } else {
         if (rows % (4 * kb) != 0 || cols % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
         if ((cols + 127) / 128 > kMaxGridY) return FP4_ERR_UNSUPPORTED_SHAPE;
@@ -172,7 +176,8 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
         if (!d.in_bf16 || !d.packed_out || !d.scales_out) return FP4_ERR_INVALID_ARG;
         if (fmt != FP4_MXFP4 && !d.global_scale) return FP4_ERR_INVALID_ARG;
         if (d.cols % (4 * kb) != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
-        if (d.rows >= kMaxRows || d.cols >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
+        if (d.rows >= kMaxRows || d.cols >= kMaxRows || ((d.rows + 127) / 128) * (d.cols / (4 * kb)) > kMaxRowTiles)
+            return FP4_ERR_UNSUPPORTED_SHAPE;
         if (d.ld % 8 != 0 || !aligned16(d.in_bf16) || !aligned16(d.packed_out) || !aligned16(d.scales_out))
             return FP4_ERR_MISALIGNED;
         if (d.global_scale && (reinterpret_cast<uintptr_t>(d.global_scale) & 3u)) return FP4_ERR_MISALIGNED;
