@@ -109,6 +109,45 @@ def test_nv_quantizer_bruteforce_sampled(orc, gs):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("gs", [1.0, 50.0 * 4.0 / 2688.0, 2.0 ** -10, 0.37, 1e-38, 3e38])
+def test_p1e8_quantizer_bruteforce_sampled(orc, gs):
+    # E8M0 block scale on 16-element blocks under S_global: S_block = 2^e with
+    # e the smallest integer such that 2^e >= max(amax / (6 gs), 1e-8) (the
+    # ratio formed in FP32), capped at 127; elements times RN(1 / (2^e gs)).
+    # The slow form below finds e with an FP64 log2 and checks both sides.
+    gs = np.float32(gs)
+    rng = np.random.default_rng(8)
+    nblk = 20000
+    amax = (2.0 ** rng.uniform(-20, 20, nblk)).astype(np.float32)
+    amax_bits = synth.f32_to_bf16_bits(amax)
+    amax_bits[:64] = synth.f32_to_bf16_bits(np.float32(6.0) * 2.0 ** np.arange(-32, 32).astype(np.float32))
+    amax = bf16_to_f32(amax_bits)
+    frac = rng.uniform(-1, 1, (nblk, 15)).astype(np.float32)
+    vals = bf16_to_f32(synth.f32_to_bf16_bits(frac * amax[:, None]))
+    vals = np.where(np.abs(vals) > amax[:, None], np.copysign(amax[:, None], vals), vals)
+    x = np.ascontiguousarray(np.concatenate([amax_bits[:, None], synth.f32_to_bf16_bits(vals)], axis=1),
+                             dtype=np.uint16)
+    packed, scales, rm = orc.quantize(orc.P1E8, orc.ROWWISE, x, gs=float(gs), with_rowmajor_scales=True)
+    xf = bf16_to_f32(x)
+    a32 = np.abs(xf).max(axis=1).astype(np.float32)
+    with np.errstate(over="ignore", divide="ignore"):
+        ratio = (a32 / (np.float32(6.0) * gs)).astype(np.float32)
+    r = np.maximum(ratio.astype(np.float64), np.float64(np.float32(1e-8)))
+    with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
+        e = np.where(np.isinf(r), 200.0, np.ceil(np.log2(r)))
+    e = np.where((e > -200) & (2.0 ** (e - 1) >= r), e - 1, e)   # smallest e with 2^e >= r
+    e = np.minimum(e, 127).astype(np.int64)
+    assert np.all((2.0 ** e.astype(np.float64) >= np.minimum(r, 2.0 ** 127)))
+    assert np.array_equal(rm[:, 0].astype(np.int64), e + 127)
+    eff = (np.ldexp(np.float32(1.0), e).astype(np.float32) * gs).astype(np.float32)
+    with np.errstate(divide="ignore", over="ignore"):
+        inv = np.where(eff == 0, np.float32(0), np.float32(1.0) / eff).astype(np.float32)
+    inv = np.minimum(inv, np.finfo(np.float32).max)
+    v = (xf * inv[:, None]).astype(np.float32)
+    want = nearest_e2m1_codes(v.ravel()).reshape(x.shape)
+    assert np.array_equal(unpack_nibbles(packed), want)
+
+
 def test_colwise_is_rowwise_of_transpose(orc):
     x = synth.normal_bf16(96, 200, seed=11, outlier_factor=20.0)
     for fmt in (orc.NVFP4, orc.MXFP4):
