@@ -63,8 +63,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_rank%d.csv" % gpu_index) \
-            if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else None
+        # raw samples are kept only when a directory for them is named
+        d = os.environ.get("FP4_BENCH_CLOCKS_DIR")
+        self.path = os.path.join(d, "clocks_rank%d.csv" % gpu_index) if d and os.path.isdir(d) else None
 
     def start(self):
         try:
