@@ -1,6 +1,7 @@
 /*
- * fp4.h -- C ABI of libfp4: microscaling FP4 quantization (NVFP4, MXFP4) and
- * the native W4A4 block-scaled GEMM on NVIDIA B200 (sm_100a).
+ * fp4.h -- C ABI of libfp4: microscaling FP4 quantization (NVFP4, MXFP4 and
+ * P1E8, one tensor or a batch), reconstruction to BF16, and the native W4A4
+ * block-scaled GEMM (single, grouped, decode) on NVIDIA B200 (sm_100a).
  *
  * The operations come from these web pages (cited by title and section):
  *  [NVFP4-Arch] "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell"
@@ -19,7 +20,10 @@
  *  - All data pointers are CUDA device pointers owned by the caller; the
  *    library never allocates or frees caller-visible memory.
  *  - Every call validates its arguments on the host first.  A call that
- *    returns anything but FP4_OK has launched nothing.  A call that returns
+ *    returns anything but FP4_OK has launched nothing, except FP4_ERR_CUDA
+ *    from a call that makes several launches (batches above 8 tensors or 16
+ *    problems, the amax pass of a dynamic quantization), where launches
+ *    before the failing one may have been queued.  A call that returns
  *    FP4_OK has queued its kernels on `stream` (asynchronous; the results are
  *    ready once the stream reaches that point).  Nothing is printed, nothing
  *    aborts the process.
@@ -31,7 +35,7 @@
  *  - Packed FP4: two E2M1 codes per byte, the even index in the low nibble,
  *    K-major rows of K/2 bytes.  Code = sign bit (bit 3) | exponent (bits 2-1)
  *    | mantissa (bit 0); values {0, 0.5, 1, 1.5, 2, 3, 4, 6} with signed zero.
- *  - Scales: one byte per block (E4M3 for NVFP4, E8M0 for MXFP4) stored in
+ *  - Scales: one byte per block (E4M3 for NVFP4, E8M0 for MXFP4 and P1E8) stored in
  *    512-byte tiles of 128 rows x 4 block-columns, tiles ordered with the
  *    block-column tile fastest; inside a tile the byte of (row r, block c) is
  *    at (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).  This is the layout the
