@@ -133,3 +133,26 @@ def test_gemm_grouped_host_checks_without_gpu():
     assert call(0, [G(0, 0, 0, 0, 0, 16, 64, None, 0, 16)]) == 0         # empty only: no-op
     if not torch.cuda.is_available():
         assert call(0, [good]) == 6
+
+
+def test_dequantize_and_dynamic_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    dq = L.fp4_dequantize
+    assert dq(7, A16, A16, A16, 16, 512, A16, 512, None) == 1          # bad format
+    assert dq(0, A16, A16, None, 16, 512, A16, 512, None) == 1         # NVFP4 without S_global
+    assert dq(0, A16, A16, A16, 16, 512, A16, 256, None) == 1          # ld < k
+    assert dq(0, A16, A16, A16, 16, 480, A16, 480, None) == 2          # k % 64
+    assert dq(1, A16, A16, None, 16, 192, A16, 192, None) == 2         # k % 128 (MX)
+    assert dq(0, A1, A16, A16, 16, 512, A16, 512, None) == 3           # misaligned packed
+    assert dq(0, A16, A16, A16, 16, 512, A16, 516, None) == 3          # ld % 8
+    assert dq(0, A16, A16, A16, 0, 512, A16, 512, None) == 0           # empty: no-op
+    dyn = L.fp4_quantize_dynamic
+    assert dyn(1, A16, 4, 128, 128, A16, A16, A16, None, None, None) == 1      # MXFP4: no S_global
+    assert dyn(0, A16, 4, 128, 128, A16, A16, None, None, None, None) == 1     # no gs_out
+    assert dyn(0, A16, 4, 128, 128, A16, A16, A16, None, A16, None) == 1       # alpha without other
+    assert dyn(0, A16, 4, 96, 96, A16, A16, A16, None, None, None) == 2        # cols % 64
+    assert dyn(0, A1, 4, 128, 128, A16, A16, A16, None, None, None) == 3       # misaligned input
+    if not torch.cuda.is_available():
+        assert dq(0, A16, A16, A16, 16, 512, A16, 512, None) == 6
+        assert dyn(0, A16, 4, 128, 128, A16, A16, A16, None, None, None) == 6
