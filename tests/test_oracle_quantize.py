@@ -307,3 +307,26 @@ def test_reconstruction_error_bound(orc):
     step = np.select([r <= 2, r <= 4], [0.5, 1.0], 2.0)
     assert np.all(r <= 6.0)
     assert np.all(np.abs(xf - deq) <= 0.5 * step * S)
+
+
+@pytest.mark.parametrize("fmt", ["nv", "mx", "p1e8"])
+def test_dequantize_is_code_times_scales(orc, fmt):
+    # x_hat = E2M1(code) * S_block (* S_global), written out here from the
+    # packed nibbles and the row-major scale bytes: E4M3 for NVFP4 (torch's
+    # FP8 decode), 2^(byte - 127) for the E8M0 formats
+    f = {"nv": orc.NVFP4, "mx": orc.MXFP4, "p1e8": orc.P1E8}[fmt]
+    k = 32 if fmt == "mx" else 16
+    x = synth.normal_bf16(40, 512, seed=18, outlier_factor=80.0, zero_frac=0.05)
+    gs = orc.global_scale(x) if fmt != "mx" else 1.0
+    p, s, rm = orc.quantize(f, orc.ROWWISE, x, gs=gs, with_rowmajor_scales=True)
+    deq = orc.dequantize(f, p, s, gs=gs if fmt != "mx" else 0.0)
+    codes = unpack_nibbles(p).astype(np.int64)
+    mags = np.array(E2M1_MAGS, dtype=np.float64)[codes & 7]
+    vals = np.where(codes & 8, -mags, mags)
+    if fmt == "nv":
+        sv = torch.from_numpy(rm.copy()).view(torch.float8_e4m3fn).double().numpy()
+    else:
+        sv = 2.0 ** (rm.astype(np.float64) - 127)
+    want = vals * np.repeat(sv, k, axis=1) * (float(np.float32(gs)) if fmt != "mx" else 1.0)
+    assert np.array_equal(deq.reshape(want.shape), want)
+    assert np.array_equal(np.signbit(deq.reshape(want.shape)), np.signbit(want))
