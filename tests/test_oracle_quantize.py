@@ -330,3 +330,40 @@ def test_dequantize_is_code_times_scales(orc, fmt):
     want = vals * np.repeat(sv, k, axis=1) * (float(np.float32(gs)) if fmt != "mx" else 1.0)
     assert np.array_equal(deq.reshape(want.shape), want)
     assert np.array_equal(np.signbit(deq.reshape(want.shape)), np.signbit(want))
+
+
+def first_index_nearest_mags(v):
+    """The emulation script's argmin rule written here: nearest magnitude,
+    the lower grid index on a tie (so ties go to the smaller magnitude)."""
+    a = np.abs(np.asarray(v, dtype=np.float32).astype(np.float64))
+    d = np.abs(a[:, None] - E2M1_MAGS[None, :])
+    return np.where(a >= 6.0, 6.0, E2M1_MAGS[d.argmin(axis=1)])
+
+
+@pytest.mark.parametrize("k", [16, 32])
+@pytest.mark.parametrize("page_tie", [False, True])
+def test_block_pow2_roundtrip_and_naive_against_slow_forms(orc, k, page_tie):
+    # the emulation script's block quantize / dequantize with power-of-two
+    # scales (zero-padded last block) and the naive per-tensor baseline,
+    # each written here from its definition
+    rng = np.random.default_rng(19)
+    x = (rng.standard_normal(1000) * 0.5).astype(np.float32)
+    x[42], x[512] = 24.5, -31.2
+    x[100:116] = 0.0
+    x[200] = 0.75 * 2.0 ** -3   # a tie point
+    got = orc.block_pow2_roundtrip(x, k, page_tie=page_tie)
+    want = np.empty(x.size)
+    for b0 in range(0, x.size, k):
+        blk = x[b0:b0 + k]
+        amax = max(float(np.abs(blk).max()), float(np.float32(1e-8)))
+        e = int(np.ceil(np.log2(amax / 6.0)))
+        if 6.0 * 2.0 ** (e - 1) >= amax:
+            e -= 1
+        v = (blk * np.float32(2.0 ** -e)).astype(np.float32)
+        mags = first_index_nearest_mags(v) if page_tie else E2M1_MAGS[nearest_e2m1_codes(v) & 7]
+        want[b0:b0 + k] = np.where(np.signbit(v), -mags, mags) * 2.0 ** e
+    assert np.array_equal(got, want)
+    s = np.float32(max(np.float32(np.abs(x).max()), np.float32(1e-8)) / np.float32(6.0))
+    v = (x / s).astype(np.float32)
+    mags = E2M1_MAGS[nearest_e2m1_codes(v) & 7]
+    assert np.array_equal(orc.naive_per_tensor(x), np.where(np.signbit(v), -mags, mags) * float(s))
