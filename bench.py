@@ -545,10 +545,14 @@ def run_reference(args):
 
     class HostOnly(SquareWorkload):
         def __init__(self):
-            self.fmt, self.n = fmt, 4096
-            self.host = synth.square(4096)
-            self.flops = 2.0 * 4096 ** 3
-            self.name = "%s quantize+GEMM M=N=K=4096" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4")
+            n, sets = 4096, 4
+            self.fmt, self.n = fmt, n
+            self.host = synth.square(n)
+            self.flops = 2.0 * n ** 3
+            self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
+            # the same config description as this workload's line on the GPU arm
+            self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
+                sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
 
     wl = HostOnly()
     # each step is a bounded sample: the whole run stays within a few minutes
@@ -565,7 +569,9 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": wl.name},
+        "data": "synthetic",
+        "config": {"workload": wl.name, "l2": wl.l2_note, "replicas": 1,
+                   "inputs": "seeded synthetic BF16 (Philox), outlier channels"},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": orc.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
