@@ -58,3 +58,17 @@ def test_single_rank_helpers():
     import bench
     assert bench.max_over_ranks(3.0) == 3.0
     assert bench.job_throughput(10.0, 1, 2.0) == 5.0
+
+
+def test_reference_arm_non_zero_rank_exits_quietly():
+    # under torchrun the reference arm runs on rank 0 only; the other ranks
+    # exit 0 without work or output
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
