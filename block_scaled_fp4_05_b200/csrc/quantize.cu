@@ -1,6 +1,8 @@
 // Block quantizer kernels: BF16 -> E2M1 codes + per-block scales (NVFP4,
-// MXFP4, and 16-element blocks with E8M0 scales under S_global), the
-// per-tensor amax for S_global, and alpha = gsA * gsB.
+// MXFP4, and 16-element blocks with E8M0 scales under S_global) for one
+// tensor or a batch (one launch over the tiles of up to 8 tensors), the
+// per-tensor amax for S_global, alpha = gsA * gsB, the one-launch dynamic
+// quantization of a small activation, and the reconstruction to BF16.
 //
 // Method: "NVFP4 Architecture: Microscaling & 4-Bit LLMs on Blackwell",
 // "1. The Dual-Level Mathematical Formulation" (S_global, S_block,j, q_i) and
