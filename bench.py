@@ -3,10 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 One step = one pass of the whole path over one batch of synthetic input.
-The default workload is the MXFP4 square case M = N = K = 4096: quantize A,
-quantize B (BF16 -> E2M1 + E8M0 block scales), then the block-scaled GEMM
-D = A_hat B_hat^T in BF16.  Other workloads (the decode, prefill and
-quantizer-sweep shapes) are selectable for measurement.
+The default workload is the largest single-GPU configuration, the NVFP4
+prefill up-projection M=8192, N=28672, K=8192: per step the activation's
+S_global and alpha, its quantization (BF16 -> E2M1 + E4M3 block scales), then
+the block-scaled GEMM D = A_hat W_hat^T in BF16 with the weights quantized
+once ahead of the steps.  Other workloads (the square 4096^3 case, decode,
+the down-projection, quantizer sweep, MoE, reconstruction) are selectable.
 
 Rank 0 prints one JSON line.  With N > 1 (torchrun) every rank runs an
 independent replica (the path does not shard across GPUs: no data-path
@@ -278,15 +280,16 @@ class SquareWorkload(Workload):
             r *= 2
         return r
 
+    def sample_note(self, r):
+        return ("S_global/quantization of %d rows of A and of B and the FP64 GEMM of the %dx%d "
+                "output block (K=%d), extrapolated to the %dx%d step" % (r, r, r, self.n, self.n, self.n))
+
     def cpu_baseline(self, orc, budget_s=20.0):
         r = self.calibrate(orc, budget_s)
         t_step, spent = self.oracle_sample(orc, r)
         return {"value": self.flops / t_step / 1e12, "unit": "TFLOP/s",
                 "cores": orc.num_threads(), "kind": "oracle",
-                "sample": "S_global/quantization of %d rows of A and of B and the FP64 GEMM of "
-                          "the %dx%d output block (K=%d), extrapolated to the %dx%d step; "
-                          "%.1f s of CPU work in the measured sample"
-                          % (r, r, r, self.n, self.n, self.n, spent)}
+                "sample": self.sample_note(r) + "; %.1f s of CPU work in the measured sample" % spent}
 
 
 class DecodeWorkload(Workload):
@@ -465,15 +468,22 @@ class DequantWorkload(Workload):
 
 
 class PrefillWorkload(Workload):
-    """NVFP4 prefill: activation S_global + quantize per step, weights
-    quantized once, D = A_hat W_hat^T on the persistent tensor-core kernel."""
+    """NVFP4 prefill: per step the activation's S_global (and alpha) and its
+    quantization, then D = A_hat W_hat^T on the persistent tensor-core kernel;
+    the weights are quantized once, ahead of the steps, and stay resident.
+    With dev=None only the host inputs exist (the reference arm)."""
+    TILE = 128   # side of the output tiles the CPU sample computes
 
     def __init__(self, M, N, K, dev, stream=None):
-        self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.M, self.N, self.K = M, N, K
         self.name = "NVFP4 prefill GEMM M=%d N=%d K=%d" % (M, N, K)
-        A, W = synth.prefill(M, N, K)
-        self.host = (A, W)
+        self.host = synth.prefill(M, N, K)
+        self.flops = 2.0 * M * N * K
+        self.l2_note = "operands %.0f MB > %d MB L2" % ((M + N) * K * 0.5625 / 1e6, L2_BYTES >> 20)
+        if dev is None:
+            return
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        A, W = self.host
         Ad, Wd = _dev_bf16(A, dev), _dev_bf16(W, dev)
         gW = fp4.global_scale(Wd)
         pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
@@ -488,19 +498,93 @@ class PrefillWorkload(Workload):
             [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, None, fp4.GEMM_PREFILL, stream)],
         ]]
         self.bufs = [(Ad, gA, al, pA, sA, pW, sW, D, gW)]
+        self.weights = (pW, sW, gW)
         torch.cuda.empty_cache()
         self.kernels = ["act_global_scale", "act_quantize", "gemm"]
         abytes = M * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, M, K)
-        self.work = {"gemm": 2.0 * M * N * K, "act_quantize": M * K * 2 + abytes,
+        self.work = {"gemm": self.flops, "act_quantize": M * K * 2 + abytes,
                      "act_global_scale": M * K * 2}
         self.bound = {"gemm": "tensor", "act_quantize": "hbm", "act_global_scale": "hbm"}
-        self.flops = 2.0 * M * N * K
         self.launches_per_step = 2 + 1 + 1 + 1
         self.dominant = "gemm"
-        self.l2_note = "operands %.0f MB > %d MB L2" % ((M + N) * K * 0.5625 / 1e6, L2_BYTES >> 20)
 
     def value(self, sec_per_step):
         return self.flops / sec_per_step / 1e12
+
+    # ---- end to end through the public API --------------------------------
+    def e2e_setup(self, dev):
+        A, _ = self.host
+        self.hA = synth.bits_to_torch(A).pin_memory()
+        self.hD = torch.empty((self.M, self.N), dtype=torch.bfloat16).pin_memory()
+        return self.hA.numel() * 2, self.hD.numel() * 2
+
+    def e2e_step(self, dev):
+        # the step's activation arrives from pinned host memory; the resident
+        # quantized weights are the layer's parameters; D goes back to the host
+        M, N, K = self.M, self.N, self.K
+        pW, sW, gW = self.weights
+        Ad = self.hA.to(dev, non_blocking=True)
+        gA = fp4.global_scale(Ad)
+        al = torch.empty(1, dtype=torch.float32, device=dev)
+        fp4.fp4_alpha_from_global_scales(gA, gW, al)
+        pA, sA = fp4.quantize(Ad, fp4.NVFP4, fp4.ROWWISE, gA)
+        D = fp4.gemm(fp4.NVFP4, pA, sA, pW, sW, K, alpha=al, kernel=fp4.GEMM_PREFILL)
+        self.hD.copy_(D, non_blocking=True)
+
+    # ---- the oracle on a bounded sample of the step ------------------------
+    def oracle_sample(self, orc, tiles, seed=0):
+        """The oracle on a sample of one step: S_global of the whole
+        activation, the quantization of the 128-row blocks of A that the
+        sampled tiles need, and the FP64 GEMM of `tiles` sampled 128x128
+        output tiles (K = full depth).  The weights' blocks are quantized
+        before the clock starts (they are resident, outside the step).
+        Returns (seconds per full step, extrapolated by the number of row
+        blocks and of output tiles; seconds spent)."""
+        A, W = self.host
+        T = self.TILE
+        nbm, nbn = self.M // T, self.N // T
+        rng = np.random.default_rng(seed)
+        tm = rng.integers(0, nbm, size=tiles)
+        tn = rng.integers(0, nbn, size=tiles)
+        if not hasattr(self, "_gW"):
+            self._gW = orc.global_scale(W)
+            self._qw = {}
+        for b in np.unique(tn):
+            if b not in self._qw:
+                self._qw[b] = orc.quantize(orc.NVFP4, 0, np.ascontiguousarray(W[b * T:(b + 1) * T]),
+                                           gs=self._gW)
+        t0 = time.perf_counter()
+        gA = orc.global_scale(A)
+        t1 = time.perf_counter()
+        qa = {b: orc.quantize(orc.NVFP4, 0, np.ascontiguousarray(A[b * T:(b + 1) * T]), gs=gA)
+              for b in np.unique(tm)}
+        t2 = time.perf_counter()
+        alpha = float(np.float32(gA) * np.float32(self._gW))
+        for i in range(tiles):
+            a, b = qa[tm[i]], self._qw[tn[i]]
+            orc.gemm(orc.NVFP4, a[0], a[1], b[0], b[1], alpha=alpha)
+        t3 = time.perf_counter()
+        t_step = ((t1 - t0) + (t2 - t1) * nbm / len(qa) + (t3 - t2) * (nbm * nbn) / tiles)
+        return t_step, t3 - t0
+
+    def calibrate(self, orc, budget_s, max_tiles=64):
+        """Tile count whose sample takes about budget_s seconds (4..max_tiles)."""
+        _, spent = self.oracle_sample(orc, 2, seed=1)
+        per_tile = max(spent / 2, 1e-3)
+        return int(max(4, min(max_tiles, budget_s / per_tile)))
+
+    def sample_note(self, tiles):
+        return ("S_global of the whole %dx%d activation, quantization of the sampled 128-row "
+                "blocks of A and the FP64 GEMM of %d sampled 128x128 output tiles (K=%d); "
+                "extrapolated to the %dx%d step by row blocks and tiles" % (
+                    self.M, self.K, tiles, self.K, self.M, self.N))
+
+    def cpu_baseline(self, orc, budget_s=20.0):
+        tiles = self.calibrate(orc, budget_s)
+        t_step, spent = self.oracle_sample(orc, tiles)
+        return {"value": self.flops / t_step / 1e12, "unit": "TFLOP/s",
+                "cores": orc.num_threads(), "kind": "oracle",
+                "sample": self.sample_note(tiles) + "; %.1f s of CPU work in the measured sample" % spent}
 
 
 def make_workload(name, dev, stream):
@@ -534,27 +618,35 @@ WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle on a bounded sample
 # ---------------------------------------------------------------------------
+def host_workload(name):
+    """The workload's host inputs only (no device), for the reference arm."""
+    if name == "prefill_up":
+        return PrefillWorkload(8192, 28672, 8192, None)
+    if name == "prefill_down":
+        return PrefillWorkload(8192, 8192, 28672, None)
+    if name in ("square_mx", "square_nv"):
+        fmt = fp4.MXFP4 if name == "square_mx" else fp4.NVFP4
+
+        class HostOnly(SquareWorkload):
+            def __init__(self):
+                n, sets = 4096, 4
+                self.fmt, self.n = fmt, n
+                self.host = synth.square(n)
+                self.flops = 2.0 * n ** 3
+                self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
+                # the same config description as this workload's line on the GPU arm
+                self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
+                    sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
+        return HostOnly()
+    raise SystemExit("the reference arm covers the prefill and square workloads")
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle as orc
-    if args.workload != "square_mx" and args.workload != "square_nv":
-        raise SystemExit("the reference arm covers the square workloads")
-    fmt = fp4.MXFP4 if args.workload == "square_mx" else fp4.NVFP4
-
-    class HostOnly(SquareWorkload):
-        def __init__(self):
-            n, sets = 4096, 4
-            self.fmt, self.n = fmt, n
-            self.host = synth.square(n)
-            self.flops = 2.0 * n ** 3
-            self.name = "%s quantize+GEMM M=N=K=%d" % ("MXFP4" if fmt == fp4.MXFP4 else "NVFP4", n)
-            # the same config description as this workload's line on the GPU arm
-            self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
-                sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
-
-    wl = HostOnly()
+    wl = host_workload(args.workload)
     # each step is a bounded sample: the whole run stays within a few minutes
     budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
     r = wl.calibrate(orc, budget)
@@ -563,8 +655,7 @@ def run_reference(args):
     secs = [wl.oracle_sample(orc, r)[0] for _ in range(args.steps)]
     sec = statistics.median(secs)
     v = wl.flops / sec / 1e12
-    sample = ("per step: S_global/quantization of %d rows of A and of B and the FP64 GEMM of "
-              "the %dx%d output block (K=4096), extrapolated to the 4096x4096 step" % (r, r, r))
+    sample = "per step: " + wl.sample_note(r)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
@@ -587,7 +678,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=None)
-    ap.add_argument("--workload", default="square_mx", choices=WORKLOADS)
+    ap.add_argument("--workload", default="prefill_up", choices=WORKLOADS)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -615,7 +706,8 @@ def main():
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.set_stream(stream)
     wl = make_workload(args.workload, dev, stream)
-    per_step_guess = {"square_mx": 60e-6, "square_nv": 70e-6}.get(args.workload, 200e-6)
+    per_step_guess = {"square_mx": 60e-6, "square_nv": 70e-6, "prefill_up": 0.9e-3,
+                      "prefill_down": 1.0e-3}.get(args.workload, 200e-6)
     steps = args.steps if args.steps is not None else max(50, int(2.0 / per_step_guess))
     warmup = args.warmup if args.warmup is not None else max(3, min(200, steps // 20))
 
