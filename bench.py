@@ -203,8 +203,8 @@ class SquareWorkload(Workload):
                 gA = torch.empty(1, dtype=torch.float32, device=dev)
                 gB = torch.empty(1, dtype=torch.float32, device=dev)
                 al = torch.empty(1, dtype=torch.float32, device=dev)
-                groups.append([fp4.bind_global_scale(Ad, gA, stream), fp4.bind_global_scale(Bd, gB, stream),
-                               fp4.bind_alpha(gA, gB, al, stream)])
+                groups.append([fp4.bind_global_scale(Ad, gA, stream),
+                               fp4.bind_global_scale_alpha(Bd, gB, gA, al, stream)])
             else:
                 gA = gB = al = None
             groups.append([fp4.bind_quantize_batch(fmt, [(Ad, pA, sA, gA), (Bd, pB, sB, gB)], stream)])
@@ -216,7 +216,7 @@ class SquareWorkload(Workload):
         self.work = {"quantize": 2 * qbytes, "gemm": 2.0 * n ** 3, "global_scales": 2.0 * n * n * 2}
         self.bound = {"quantize": "hbm", "gemm": "tensor", "global_scales": "hbm"}
         self.flops = 2.0 * n ** 3
-        self.launches_per_step = 2 if fmt == fp4.MXFP4 else 2 + 2 * 2 + 1
+        self.launches_per_step = 2 if fmt == fp4.MXFP4 else 4
         self.dominant = "gemm"
         self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
             sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
@@ -236,9 +236,10 @@ class SquareWorkload(Workload):
         Ad = self.hA.to(dev, non_blocking=True)
         Bd = self.hB.to(dev, non_blocking=True)
         if fmt == fp4.NVFP4:
-            gA, gB = fp4.global_scale(Ad), fp4.global_scale(Bd)
+            gA = fp4.global_scale(Ad)
+            gB = torch.empty(1, dtype=torch.float32, device=dev)
             al = torch.empty(1, dtype=torch.float32, device=dev)
-            fp4.fp4_alpha_from_global_scales(gA, gB, al)
+            fp4.fp4_compute_global_scale_alpha(Bd, gB, gA, al)
         else:
             gA = gB = al = None
         pA, sA = _qbufs(fmt, n, n, dev)
@@ -492,20 +493,21 @@ class PrefillWorkload(Workload):
         al = torch.empty(1, dtype=torch.float32, device=dev)
         pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
         D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        # per step: the activation's S_global and alpha (one launch), its
+        # quantization (one launch), the GEMM
         self.calls = [[
-            [fp4.bind_global_scale(Ad, gA, stream), fp4.bind_alpha(gA, gW, al, stream)],
-            [fp4.bind_quantize(fp4.NVFP4, fp4.ROWWISE, Ad, pA, sA, gA, stream)],
+            [fp4.bind_quantize_dynamic(Ad, pA, sA, gA, gW, al, stream)],
             [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, None, fp4.GEMM_PREFILL, stream)],
         ]]
         self.bufs = [(Ad, gA, al, pA, sA, pW, sW, D, gW)]
         self.weights = (pW, sW, gW)
         torch.cuda.empty_cache()
-        self.kernels = ["act_global_scale", "act_quantize", "gemm"]
+        self.kernels = ["act_quantize", "gemm"]
         abytes = M * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, M, K)
-        self.work = {"gemm": self.flops, "act_quantize": M * K * 2 + abytes,
-                     "act_global_scale": M * K * 2}
-        self.bound = {"gemm": "tensor", "act_quantize": "hbm", "act_global_scale": "hbm"}
-        self.launches_per_step = 2 + 1 + 1 + 1
+        # two passes over the activation (amax, then quantization) + codes and scales
+        self.work = {"gemm": self.flops, "act_quantize": 2 * M * K * 2 + abytes}
+        self.bound = {"gemm": "tensor", "act_quantize": "hbm"}
+        self.launches_per_step = 3
         self.dominant = "gemm"
 
     def value(self, sec_per_step):
@@ -524,10 +526,10 @@ class PrefillWorkload(Workload):
         M, N, K = self.M, self.N, self.K
         pW, sW, gW = self.weights
         Ad = self.hA.to(dev, non_blocking=True)
-        gA = fp4.global_scale(Ad)
+        gA = torch.empty(1, dtype=torch.float32, device=dev)
         al = torch.empty(1, dtype=torch.float32, device=dev)
-        fp4.fp4_alpha_from_global_scales(gA, gW, al)
-        pA, sA = fp4.quantize(Ad, fp4.NVFP4, fp4.ROWWISE, gA)
+        pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
+        fp4.fp4_quantize_dynamic(Ad, pA, sA, gA, gW, al)
         D = fp4.gemm(fp4.NVFP4, pA, sA, pW, sW, K, alpha=al, kernel=fp4.GEMM_PREFILL)
         self.hD.copy_(D, non_blocking=True)
 

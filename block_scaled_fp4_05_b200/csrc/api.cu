@@ -81,7 +81,7 @@ constexpr int64_t kMaxRowTiles = (int64_t)1 << 28;
 
 extern "C" {
 
-int fp4_abi_version(void) { return 2; }
+int fp4_abi_version(void) { return 3; }
 
 const char* fp4_last_error(void) { return fp4::g_last_error; }
 
@@ -126,8 +126,30 @@ fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t c
     fp4::DeviceInfo dev;
     fp4_status st = require_device(&dev);
     if (st != FP4_OK) return st;
-    return from_cuda(fp4::launch_amax(static_cast<const uint16_t*>(in_bf16), rows, cols, ld, gs_out,
-                                      reinterpret_cast<cudaStream_t>(stream)));
+    return from_cuda(fp4::launch_global_scale(static_cast<const uint16_t*>(in_bf16), rows, cols, ld,
+                                              gs_out, nullptr, nullptr,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4_status fp4_compute_global_scale_alpha(const void* in_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                          float* gs_out, const float* other_gs, float* alpha_out,
+                                          fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (rows < 0 || cols < 0 || gs_out == nullptr || other_gs == nullptr || alpha_out == nullptr)
+        return FP4_ERR_INVALID_ARG;
+    if (rows > 0 && cols > 0 && in_bf16 == nullptr) return FP4_ERR_INVALID_ARG;
+    if (ld < cols) return FP4_ERR_INVALID_ARG;
+    if (cols % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld % 8 != 0 || !aligned16(in_bf16) || (reinterpret_cast<uintptr_t>(gs_out) & 3u) ||
+        (reinterpret_cast<uintptr_t>(other_gs) & 3u) || (reinterpret_cast<uintptr_t>(alpha_out) & 3u))
+        return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_global_scale(static_cast<const uint16_t*>(in_bf16), rows, cols, ld,
+                                              gs_out, other_gs, alpha_out,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int64_t rows,

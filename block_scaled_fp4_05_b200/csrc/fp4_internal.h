@@ -24,8 +24,11 @@ struct DeviceInfo {
 cudaError_t device_info(DeviceInfo* out);
 
 // quantize.cu
-cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                        float* gs_out, cudaStream_t s);
+// S_global of x (and alpha = S_global * *other_gs when alpha_out is set) in
+// one launch.
+cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                float* gs_out, const float* other_gs, float* alpha_out,
+                                cudaStream_t s);
 cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s);
 cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                                     uint8_t* packed, uint8_t* scales, float* gs_out,
@@ -43,7 +46,9 @@ struct RowwiseDesc {
     uint8_t* scales;
     const float* gs;   // NVFP4 S_global, NULL for MXFP4
 };
-cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s);
+// reverse: the tiles run last to first (same results).
+cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s,
+                                          bool reverse = false);
 
 // gemm.cu
 struct GemmArgs {

@@ -23,6 +23,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 #include <cfloat>
+#include <mutex>
 
 #include "fp4_internal.h"
 
@@ -198,6 +199,7 @@ __device__ __forceinline__ void rowwise_tile(const uint16_t* __restrict__ x, int
 // fastest.  Used by both rowwise kernels (with their own tile widths).
 struct RowBatch {
     int n;
+    int reverse;                         // tiles in reverse order (last tile first)
     int64_t tile_begin[kMaxBatch + 1];   // prefix sums of the tensors' tile counts
     const uint16_t* x[kMaxBatch];
     int64_t rows[kMaxBatch], cols[kMaxBatch], ld[kMaxBatch];
@@ -227,7 +229,7 @@ quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
     constexpr int TILE_C = 4 * (FMT == kMx ? 32 : 16);
     int k;
     int64_t rt, ct;
-    locate_tile(b, blockIdx.x, TILE_C, k, rt, ct);
+    locate_tile(b, b.reverse ? gridDim.x - 1 - blockIdx.x : blockIdx.x, TILE_C, k, rt, ct);
     float gs = 1.0f, denom = 6.0f;
     if (FMT != kMx) {
         gs = __ldg(b.gs[k]);
@@ -535,32 +537,48 @@ quantize_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
 }
 
 // ---------------------------------------------------------------------------
-// amax over a BF16 matrix into a 32-bit word (BF16 magnitude bits), then
-// S_global = amax / 2688 (1 when amax == 0) in place.
+// S_global = amax / 2688 (1 when amax == 0) of a BF16 matrix, and optionally
+// alpha = S_global * other, in one launch.  Each CTA reduces its share of the
+// rows to one BF16 magnitude (an integer max over the magnitude bits) and
+// folds it into a reduction slot with atomicMax; the CTA whose arrival on the
+// slot's counter is the last one finalizes: it reads the slot's maximum,
+// writes S_global (and alpha) and resets the slot to zero for its next use.
+// The slots live in a ring in static device memory, zero at load; each call
+// takes the next slot, so calls in flight at the same time (other streams)
+// reduce into different slots.
 // ---------------------------------------------------------------------------
+struct GsSlot {
+    unsigned int amax;    // BF16 magnitude bits
+    unsigned int count;   // CTAs arrived
+};
+constexpr int kGsSlots = 1024;
+__device__ GsSlot g_gs_slots[kGsSlots];
+
+constexpr int kGsUnroll = 4;   // 16-byte loads in flight per thread
+
+// Rows are split into segments of kThreads * kGsUnroll chunks (8 BF16 each);
+// the CTAs take segments in a grid-stride loop, so no per-load index
+// division is needed.  A contiguous matrix (ld == cols) is one long row.
 __global__ void __launch_bounds__(kThreads)
-amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld,
-            unsigned int* __restrict__ word)
+global_scale_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cpr, int64_t ld,
+                    int64_t segs_per_row, GsSlot* __restrict__ slot, float* __restrict__ gs_out,
+                    const float* __restrict__ other_gs, float* __restrict__ alpha_out)
 {
-    const int64_t cpr = cols / 8;
-    const int64_t total = rows * cpr;
+    pdl_trigger();
+    const int64_t total = rows * segs_per_row;
     uint32_t m = 0;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    for (; i + 3 * stride < total; i += 4 * stride) {
-        uint4 v[4];
+    for (int64_t sidx = blockIdx.x; sidx < total; sidx += gridDim.x) {
+        const int64_t r = sidx / segs_per_row;
+        const int64_t c0 = (sidx - r * segs_per_row) * (kThreads * kGsUnroll) + threadIdx.x;
+        const uint4* row = reinterpret_cast<const uint4*>(x + r * ld);
+        uint4 v[kGsUnroll];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t j = i + u * stride;
-            const int64_t r = j / cpr, c = j % cpr;
-            v[u] = ld_stream(reinterpret_cast<const uint4*>(x + r * ld) + c);
+        for (int u = 0; u < kGsUnroll; ++u) {
+            const int64_t c = c0 + u * kThreads;
+            v[u] = c < cpr ? ld_stream(row + c) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) m = max(m, absmax8(v[u]));
-    }
-    for (; i < total; i += stride) {
-        const int64_t r = i / cpr, c = i % cpr;
-        m = max(m, absmax8(ld_stream(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+        for (int u = 0; u < kGsUnroll; ++u) m = max(m, absmax8(v[u]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -570,15 +588,23 @@ amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t 
     if (threadIdx.x == 0) {
         uint32_t b = 0;
         for (int w = 0; w < kThreads / 32; ++w) b = max(b, s_m[w]);
-        if (b) atomicMax(word, b);
+        if (b) atomicMax(&slot->amax, b);
+        // release: this CTA's maximum is visible before its arrival counts;
+        // acquire: the last arriver sees every other CTA's maximum
+        unsigned int old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(old) : "l"(&slot->count) : "memory");
+        if (old == gridDim.x - 1) {
+            unsigned int bits;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(&slot->amax) : "memory");
+            const float amax = __uint_as_float(bits << 16);
+            const float gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+            *gs_out = gs;
+            if (alpha_out) *alpha_out = __fmul_rn(gs, *other_gs);
+            slot->amax = 0u;
+            slot->count = 0u;
+        }
     }
-}
-
-__global__ void global_scale_finalize_kernel(float* gs)
-{
-    const unsigned int bits = *reinterpret_cast<unsigned int*>(gs);
-    const float amax = __uint_as_float(bits << 16);
-    *gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
 }
 
 __global__ void alpha_kernel(const float* a, const float* b, float* out)
@@ -586,29 +612,26 @@ __global__ void alpha_kernel(const float* a, const float* b, float* out)
     *out = __fmul_rn(*a, *b);
 }
 
-}  // namespace
-
-cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, float* gs_out,
-                        cudaStream_t s)
+// Device address of the slot ring on the current device (looked up once per
+// device: in host code the array's name is not a device address).
+cudaError_t gs_slots(GsSlot** out)
 {
-    cudaError_t e = cudaMemsetAsync(gs_out, 0, sizeof(float), s);
+    static std::mutex mu;
+    static GsSlot* cache[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    const int64_t chunks = rows * (cols / 8);
-    if (chunks > 0) {
-        DeviceInfo dev;
-        e = device_info(&dev);
-        if (e != cudaSuccess) return e;
-        int64_t grid = (chunks + kThreads - 1) / kThreads;
-        const int64_t cap = (int64_t)dev.sm_count * 8;
-        if (grid > cap) grid = cap;
-        amax_kernel<<<(unsigned)grid, kThreads, 0, s>>>(x, rows, cols, ld,
-                                                       reinterpret_cast<unsigned int*>(gs_out));
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) {
+        *out = cache[dev];
+        return cudaSuccess;
     }
-    global_scale_finalize_kernel<<<1, 1, 0, s>>>(gs_out);
-    return cudaGetLastError();
+    e = cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_gs_slots);
+    if (e == cudaSuccess && dev < 64) cache[dev] = *out;
+    return e;
 }
+
+}  // namespace
 
 cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s)
 {
@@ -616,14 +639,48 @@ cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaS
     return cudaGetLastError();
 }
 
+cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                float* gs_out, const float* other_gs, float* alpha_out,
+                                cudaStream_t s)
+{
+    static unsigned int next_slot = 0;   // ring position (atomic: calls from several threads)
+    DeviceInfo dev;
+    cudaError_t e = device_info(&dev);
+    if (e != cudaSuccess) return e;
+    GsSlot* slots = nullptr;
+    e = gs_slots(&slots);
+    if (e != cudaSuccess) return e;
+    const unsigned int k = __atomic_fetch_add(&next_slot, 1u, __ATOMIC_RELAXED) % kGsSlots;
+    // a contiguous matrix is reduced as one row
+    const bool flat = ld == cols;
+    const int64_t r = flat ? 1 : rows;
+    const int64_t cpr = flat ? rows * cols / 8 : cols / 8;
+    const int64_t spr = (cpr + kThreads * kGsUnroll - 1) / (kThreads * kGsUnroll);
+    int64_t grid = r * spr;
+    const int64_t cap = (int64_t)dev.sm_count * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    global_scale_kernel<<<(unsigned)grid, kThreads, 0, s>>>(x, r, cpr, ld, spr, slots + k, gs_out,
+                                                            other_gs, alpha_out);
+    return cudaGetLastError();
+}
+
 namespace {
 
 // Cluster size for the dynamic quantizer: 16 CTAs when the device can place
-// such a cluster, else the portable 8.  Decided once per process.
+// such a cluster, else the portable 8.  Decided once per device (the
+// non-portable-size attribute is set on each device that uses it).
 int dynamic_cluster_size()
 {
-    static int size = 0;
-    if (size) return size;
+    static std::mutex mu;
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return kDynClusterMin;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) return cache[dev];
     int chosen = kDynClusterMin;
     if (cudaFuncSetAttribute(quantize_dynamic_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
         cudaSuccess) {
@@ -642,8 +699,8 @@ int dynamic_cluster_size()
             chosen = kDynClusterMax;
     }
     cudaGetLastError();
-    size = chosen;
-    return size;
+    if (dev < 64) cache[dev] = chosen;
+    return chosen;
 }
 
 }  // namespace
@@ -654,11 +711,13 @@ cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t col
 {
     const int cl = dynamic_cluster_size();
     if (rows * (cols / 8) > (int64_t)cl * kDynThreads * kDynRegChunks) {
-        // too large to stay in one cluster's registers: amax pass, then the
-        // rowwise quantizer and alpha as separate kernels
-        cudaError_t e = launch_amax(x, rows, cols, ld, gs_out, s);
-        if (e == cudaSuccess) e = launch_quantize(kNv, 0, x, rows, cols, ld, packed, scales, gs_out, s);
-        if (e == cudaSuccess && alpha_out) e = launch_alpha(gs_out, other_gs, alpha_out, s);
+        // too large to stay in one cluster's registers: S_global and alpha in
+        // one launch, then the rowwise quantizer.  The quantizer takes its
+        // tiles in reverse order: the amax pass ends at the tensor's last rows,
+        // so those are still in L2 when the quantizer starts on them.
+        cudaError_t e = launch_global_scale(x, rows, cols, ld, gs_out, other_gs, alpha_out, s);
+        const RowwiseDesc d = {x, rows, cols, ld, packed, scales, gs_out};
+        if (e == cudaSuccess) e = launch_quantize_rowwise_batch(kNv, 1, &d, s, true);
         if (e != cudaSuccess) set_last_error("dynamic quantizer (multi-kernel) launch", e);
         return e;
     }
@@ -684,12 +743,14 @@ cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t col
 // variant that streamed the tiles through a cp.async ring in shared memory
 // was measured slower for both formats: one CTA per tile, many of them
 // resident, keeps more loads in flight.)
-cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s)
+cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, cudaStream_t s,
+                                          bool reverse)
 {
     const int64_t tile_c = 4 * block_size(fmt);
     for (int i0 = 0; i0 < n; i0 += kMaxBatch) {
         RowBatch b = {};
         b.n = 0;
+        b.reverse = reverse ? 1 : 0;
         b.tile_begin[0] = 0;
         for (int i = i0; i < n && i < i0 + kMaxBatch; ++i) {
             if (d[i].rows == 0 || d[i].cols == 0) continue;

@@ -60,6 +60,8 @@ def lib():
         L.fp4_scale_bytes.argtypes = [c.c_int, i64, i64]
         L.fp4_compute_global_scale.restype = c.c_int
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
+        L.fp4_compute_global_scale_alpha.restype = c.c_int
+        L.fp4_compute_global_scale_alpha.argtypes = [P, i64, i64, i64, P, P, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
         L.fp4_gemm_grouped.restype = c.c_int
@@ -146,6 +148,16 @@ def fp4_compute_global_scale(x, gs_out, stream=None):
     _check(lib().fp4_compute_global_scale(_dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
                                           _dptr(gs_out, "gs_out"), _stream(stream)),
            "fp4_compute_global_scale")
+
+
+def fp4_compute_global_scale_alpha(x, gs_out, other_gs, alpha_out, stream=None):
+    """S_global of x into gs_out and alpha = S_global * other_gs into alpha_out
+    (float32 CUDA tensors of 1 element), one launch."""
+    assert x.dtype == torch.bfloat16 and gs_out.dtype == torch.float32
+    _check(lib().fp4_compute_global_scale_alpha(_dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                                                _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"),
+                                                _dptr(alpha_out, "alpha_out"), _stream(stream)),
+           "fp4_compute_global_scale_alpha")
 
 
 def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):
@@ -339,6 +351,12 @@ class BoundCall:
 def bind_global_scale(x, gs_out, stream=None):
     return BoundCall("fp4_compute_global_scale", _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
                      _dptr(gs_out, "gs_out"), _stream(stream))
+
+
+def bind_global_scale_alpha(x, gs_out, other_gs, alpha_out, stream=None):
+    return BoundCall("fp4_compute_global_scale_alpha", _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
+                     _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"), _dptr(alpha_out, "alpha_out"),
+                     _stream(stream))
 
 
 def bind_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):

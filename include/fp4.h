@@ -129,10 +129,26 @@ size_t fp4_scale_bytes(fp4_format fmt, int64_t rows, int64_t k);
  * reading of its precision).
  *   in_bf16 : device, rows x cols, leading dimension ld (elements)
  *   gs_out  : device, one float, written asynchronously
- * Requires cols % 8 == 0.
+ * Requires cols % 8 == 0.  One launch: the CTAs reduce their rows, the last
+ * one to finish writes S_global.  Its partial maxima meet in one of 1024
+ * reduction slots in the library's static device memory, taken in turn by
+ * successive calls and left zeroed by each call, so up to 1024 calls may be
+ * in flight at once (on any streams) without sharing a slot.  A call captured
+ * in a CUDA graph keeps its slot in every replay of the graph.
  */
 fp4_status fp4_compute_global_scale(const void* in_bf16, int64_t rows, int64_t cols,
                                     int64_t ld, float* gs_out, fp4_stream_t stream);
+
+/*
+ * fp4_compute_global_scale followed by alpha = S_global * (*other_gs) (the
+ * product fp4_alpha_from_global_scales forms), both in the same single
+ * launch: the two per-tensor factors of an NVFP4 GEMM whose other operand's
+ * S_global is already known.  gs_out, other_gs and alpha_out are device
+ * floats (other_gs written by earlier work on the stream, or constant).
+ */
+fp4_status fp4_compute_global_scale_alpha(const void* in_bf16, int64_t rows, int64_t cols,
+                                          int64_t ld, float* gs_out, const float* other_gs,
+                                          float* alpha_out, fp4_stream_t stream);
 
 /*
  * Block quantization BF16 -> E2M1 codes + one scale per block.
@@ -214,8 +230,10 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
  * identical to those three calls.  One cluster of 16 CTAs (8 where the device
  * cannot place 16) holds the tensor in registers between the amax and the
  * quantization; a tensor above that capacity (65536 16-byte chunks, i.e.
- * 1 MiB of BF16, with 16 CTAs) is handled inside the same call by the
- * separate amax, quantize and alpha kernels.
+ * 1 MiB of BF16, with 16 CTAs) is handled inside the same call by two
+ * launches: S_global and alpha (as fp4_compute_global_scale_alpha), then the
+ * rowwise quantizer, which visits the tensor's tiles last to first so that
+ * the rows the first pass read last are still in L2.
  *   fmt      : FP4_NVFP4 only (MXFP4 needs no per-tensor scale: use
  *              fp4_quantize); else FP4_ERR_INVALID_ARG
  *   in_bf16  : device, rows x cols (ld), cols % 64 == 0, rows, cols > 0

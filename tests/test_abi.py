@@ -13,7 +13,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.fp4_abi_version() == 2
+    assert L.fp4_abi_version() == 3
 
 
 def test_status_strings():
@@ -156,3 +156,18 @@ def test_dequantize_and_dynamic_host_checks_without_gpu():
     if not torch.cuda.is_available():
         assert dq(0, A16, A16, A16, 16, 512, A16, 512, None) == 6
         assert dyn(0, A16, 4, 128, 128, A16, A16, A16, None, None, None) == 6
+
+
+def test_global_scale_alpha_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    f = L.fp4_compute_global_scale_alpha
+    assert f(A16, 4, 8, 8, A16, None, A16, None) == 1        # no other_gs
+    assert f(A16, 4, 8, 8, A16, A16, None, None) == 1        # no alpha_out
+    assert f(A16, 4, 8, 8, None, A16, A16, None) == 1        # no gs_out
+    assert f(A16, 4, 8, 4, A16, A16, A16, None) == 1         # ld < cols
+    assert f(A16, 4, 12, 12, A16, A16, A16, None) == 2       # cols % 8
+    assert f(A1, 4, 8, 8, A16, A16, A16, None) == 3          # misaligned input
+    assert f(A16, 4, 8, 8, A16, A16, P((1 << 20) + 2), None) == 3   # misaligned alpha
+    if not torch.cuda.is_available():
+        assert f(A16, 4, 8, 8, A16, A16, A16, None) == 6

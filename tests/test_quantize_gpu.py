@@ -128,6 +128,36 @@ def test_global_scale_with_leading_dimension(orc):
     assert np.float32(gs.item()) == np.float32(orc.global_scale(x))
 
 
+def test_global_scale_alpha_one_launch(orc):
+    # S_global and alpha = S_global * other from one launch, on a strided view
+    x = synth.normal_bf16(100, 256, seed=29, outlier_factor=30.0)
+    big = np.zeros((100, 264), dtype=np.uint16)
+    big[:, :256] = x
+    d = to_dev_bf16(big)
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    al = torch.empty(1, dtype=torch.float32, device="cuda")
+    other = to_dev_f32(0.0371)
+    fp4.fp4_compute_global_scale_alpha(d[:, :256], gs, other, al)
+    torch.cuda.synchronize()
+    g = orc.global_scale(x)
+    assert np.float32(gs.item()) == np.float32(g)
+    assert np.float32(al.item()) == np.float32(g) * np.float32(0.0371)
+
+
+def test_global_scale_slot_ring_wraps(orc):
+    # more calls than reduction slots, alternating two tensors: every call
+    # leaves its slot zeroed, so the second use of each slot is exact again
+    xs = [synth.normal_bf16(64, 512, seed=30, tensor_id=t, outlier_factor=20.0) for t in range(2)]
+    want = [np.float32(orc.global_scale(x)) for x in xs]
+    ds = [to_dev_bf16(x) for x in xs]
+    out = torch.empty(1100, dtype=torch.float32, device="cuda")
+    for i in range(1100):
+        fp4.fp4_compute_global_scale(ds[i % 2], out[i:i + 1])
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    assert np.all(got[0::2] == want[0]) and np.all(got[1::2] == want[1])
+
+
 def test_alpha_from_global_scales():
     a, b = to_dev_f32(0.0123), to_dev_f32(3.7)
     out = torch.empty(1, dtype=torch.float32, device="cuda")
@@ -182,10 +212,11 @@ def test_full_size_sweep_sampled_p1e8(orc, axis):
 
 
 @pytest.mark.parametrize("shape", [(1, 8192), (4, 8192), (16, 8192), (16, 512), (3, 64), (1, 64),
-                                   (200, 1024), (33, 8192), (300, 1024)])
+                                   (200, 1024), (33, 8192), (300, 1024), (2048, 8192)])
 def test_dynamic_quantize_matches_oracle(orc, shape):
     # one call: S_global, quantization with it, alpha = S_global * other; small tensors
-    # take the single-launch cluster kernel, (33, 8192) and (300, 1024) the multi-kernel path
+    # take the single-launch cluster kernel, (33, 8192), (300, 1024) and (2048, 8192) the
+    # two-launch path (S_global + alpha, then the quantizer over the tiles in reverse order)
     x = synth.normal_bf16(*shape, seed=28, outlier_factor=100.0)
     rows, cols = shape
     xd = to_dev_bf16(x)
