@@ -142,6 +142,20 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
@@ -900,26 +914,40 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // computes a 256 x 256 tile with tcgen05.mma.cta_group::2: each CTA stages
 // its own 128 rows of A and its half (128 rows) of the 256-row B tile, so a
 // CTA moves 32 KB of operands per 256-deep stage instead of 48 KB for the
-// same tensor work, and five stages fit in shared memory.  Each CTA keeps
-// the scales of its own A rows and of all 256 B rows in its own TMEM and
-// accumulates its 128 x 256 half of the tile there.
-//   - Both producers' A/B tensor loads complete on the leader's (rank 0)
-//     full[s] barrier; the leader's producer posts the expected bytes of
-//     both CTAs.  Scale chunks complete on each CTA's own sf_full[s].
-//   - Scale-staging warps of both CTAs arrive on the leader's sf_ready[s].
-//   - The leader's MMA thread issues the pair MMAs and releases stage s in
-//     both CTAs (and publishes the accumulator to both) with one commit
-//     that arrives on the barrier at the same offset in each CTA.
-//   - Epilogue warps of both CTAs arrive on the leader's acc_empty.
+// same tensor work.  Each CTA keeps the scales of its own A rows and of all
+// 256 B rows in its own TMEM and accumulates its 128 x 256 half of the tile
+// there.
+//   warp 0        producer: lane 0 runs the stage loop and issues the
+//                 tensor loads of A and B (both CTAs' loads
+//                 complete on the leader's (rank 0) full[s]; the leader posts
+//                 the expected bytes of both) and the scale chunks (on the
+//                 CTA's own sf_full[s]).
+//   warp 1        MMA issue (leader CTA only): lane 0 issues the pair MMAs
+//                 and releases each stage in both CTAs (and publishes the
+//                 accumulator to both) with one commit that arrives on the
+//                 barrier at the same offset in each CTA.  One barrier probe
+//                 per stage, made while the stage's MMAs run.
+//   warps 2-5, 10-13  epilogue: two warps per TMEM lane quadrant, each
+//                 draining 128 of the 256 accumulator columns (tcgen05.ld,
+//                 alpha, BF16), releasing the accumulator on the leader's
+//                 acc_empty, then storing D through shared memory with TMA.
+//   warps 6-9     scale staging: copy the stage's scale chunks into their
+//                 TMEM lane quadrant with tcgen05.st, then arrive on the
+//                 leader's full[s], so that full[s] completes when the
+//                 operands of both CTAs have landed and both CTAs' scales are
+//                 in TMEM.
+// In the producer and MMA warps the other 31 lanes wait at __syncwarp (not at
+// a warp-aligned barrier) while lane 0 runs the loop.
 // All waits are bounded; a CTA that gives up records the error, and both
 // CTAs meet at a final cluster barrier before the pair frees its TMEM.
 // ------------------------------------------------------------------------
 constexpr int PAIR_BN = 256;                 // N of the pair tile
 constexpr int PAIR_BHALF = PAIR_BN / 2;      // B rows staged by each CTA
+constexpr int kPairThreads = 448;            // 14 warps, roles above
+constexpr int kEpiWarps = 8;
 
 // Per stage, NVFP4 carries 4 scale chunks per 128 rows (one per K=64 MMA),
-// MXFP4 2 (one per two MMAs); the scale region of a stage is sized for its
-// format, so MXFP4 fits a sixth stage.
+// MXFP4 2 (one per two MMAs).
 template <int STAGES, bool MX>
 struct PairCfg {
     static constexpr int NCH = MX ? 2 : 4;                          // scale chunks per 128 rows
@@ -935,12 +963,15 @@ struct PairCfg {
     static constexpr int SFA_COLS = 4 * NCH;
     static constexpr int SF_COLS = SFA_COLS + 8 * NCH;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int NBARS = 5 * STAGES + 4;
+    static constexpr int NBARS = 3 * STAGES + 3;
+    // arrivals that complete full[s] on the leader: the producer's
+    // expect-tx arrival and the 4 scale-staging warps of each CTA
+    static constexpr int FULL_ARRIVALS = 1 + 8;
     // epilogue staging: per epilogue warp one 32-row x 32-column BF16 block
     // (64-byte rows, 64-byte swizzle) that a TMA store writes to D
     static constexpr int EPI_BLOCK = 32 * 64;
     static constexpr int OFF_EPI = STAGES * STAGE_BYTES;
-    static constexpr int OFF_BARS = OFF_EPI + 4 * EPI_BLOCK;
+    static constexpr int OFF_BARS = OFF_EPI + kEpiWarps * EPI_BLOCK;
     static constexpr int SMEM = OFF_BARS + 1024 + 512;
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
     static_assert(NBARS * 8 + 8 <= 512, "barrier area");
@@ -982,9 +1013,9 @@ __device__ __forceinline__ void cluster_sync()
 }
 
 // Arrive on a barrier of the other CTA without a cluster-scope release
-// fence.  Used only after tcgen05.wait::st, which already guarantees that the
-// tensor-memory writes the arrival announces have completed; the
-// cluster-scope release would cost ~1000 cycles per arrival.
+// fence.  Used only after tcgen05.wait::st / wait::ld, which already
+// guarantee that the tensor-memory accesses the arrival announces have
+// completed; the cluster-scope release would cost ~1000 cycles per arrival.
 __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
@@ -1004,7 +1035,7 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_
 }
 
 // Arrive on the barrier at offset `bar` in both CTAs of the pair once the
-// pair MMAs issued so far have completed.
+// pair MMAs issued so far (by this thread) have completed.
 __device__ __forceinline__ void tc_commit_pair_both(uint32_t bar)
 {
     asm volatile(
@@ -1053,6 +1084,39 @@ __device__ __forceinline__ void spin_ns(uint64_t ns)
     }
 }
 
+// Warp-uniform bounded wait, called by all 32 lanes of a warp: every lane
+// polls and the warp leaves together.  Gives up (false) when the CTA's abort
+// flag is raised or after kTimeoutNs, in which case it raises the flag and
+// records `code` in the device error word.
+__device__ __noinline__ bool warp_wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                            unsigned code)
+{
+    const uint64_t t0 = now_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+        if ((it & 15u) == 0) {
+            int give_up = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (*abort_flag) {
+                    give_up = 1;
+                } else if (now_ns() - t0 > kTimeoutNs) {
+                    *abort_flag = 1;
+                    atomicOr(&g_fp4_error_word, code);
+                    give_up = 1;
+                }
+            }
+            if (__shfl_sync(0xFFFFFFFFu, give_up, 0)) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned code)
+{
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+    return warp_wait_slow(bar, parity, abort_flag, code);
+}
+
 // The problems one pair-kernel launch computes: NG = 1 for fp4_gemm, up to
 // kMaxGroups for fp4_gemm_grouped.  Tile t of the launch belongs to problem g
 // with tile_begin[g] <= t < tile_begin[g + 1]; within a problem, M tiles
@@ -1068,7 +1132,7 @@ struct PairArgs {
 };
 
 template <int STAGES, bool MX, int NG>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kPairThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
 {
     using C = PairCfg<STAGES, MX>;
@@ -1076,8 +1140,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
-    // [0,S) full (leader), [S,2S) empty, [2S,3S) sf_full, [3S,4S) sf_ready (leader),
-    // [4S] acc_full, [4S+1] acc_empty (leader), [4S+2] drain
+    // [0,S) full (leader), [S,2S) empty, [2S,3S) sf_full,
+    // [3S] acc_full, [3S+1] acc_empty (leader), [3S+2] drain
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -1090,20 +1154,18 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
     auto B_FULL = [&](int s) { return bar0 + 8u * s; };
     auto B_EMPTY = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto B_SFFULL = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
-    auto B_SFREADY = [&](int s) { return bar0 + 8u * (3 * STAGES + s); };
-    const uint32_t acc_full = bar0 + 8u * (4 * STAGES);
-    const uint32_t acc_empty = bar0 + 8u * (4 * STAGES + 1);
-    const uint32_t drain = bar0 + 8u * (4 * STAGES + 2);
+    const uint32_t acc_full = bar0 + 8u * (3 * STAGES);
+    const uint32_t acc_empty = bar0 + 8u * (3 * STAGES + 1);
+    const uint32_t drain = bar0 + 8u * (3 * STAGES + 2);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(B_FULL(s), 1);
+            mbar_init(B_FULL(s), C::FULL_ARRIVALS);
             mbar_init(B_EMPTY(s), 1);
             mbar_init(B_SFFULL(s), 1);
-            mbar_init(B_SFREADY(s), 8);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 8);
+        mbar_init(acc_empty, 2 * kEpiWarps);
         mbar_init(drain, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1133,7 +1195,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
     };
 
     if (warp == 0) {
-        // ---------------- TMA producer (both CTAs) ----------------
+        // ---------------- producer (both CTAs, lane 0) ----------------
         if (lane == 0) {
             for (int g = 0; g < args.n; ++g) {
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&args.a[g])) : "memory");
@@ -1192,9 +1254,19 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             // CTAs meet at the final cluster barrier.
             if (!ok || *abort_flag) spin_ns(200000);
         }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer (leader CTA only) ----------------
-        if (lane == 0 && leader) {
+        // ---------------- MMA issue (leader CTA only, lane 0) ----------------
+        // The tensor pipe takes a new MMA only shortly before the previous
+        // one ends, so any work of the issuing thread between two MMAs beyond
+        // about one MMA's duration leaves the pipe idle.  The per-stage work
+        // is therefore spread over the gaps between a stage's MMAs, where the
+        // thread would wait for the pipe anyway: after MMA 0 the release of
+        // the previous stage (its commit then also covers MMA 0, releasing
+        // the slot one MMA later), after MMA 1 a non-blocking probe of the
+        // next stage's barrier; between stages only the probe's result is
+        // tested (a blocking wait only if the data is late).
+        if (leader && lane == 0) {
             const uint64_t adesc0 = desc_sw128(smem0);
             const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
             constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;
@@ -1204,63 +1276,74 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
+            int pending = -1;   // stage whose release commit is still to be issued
             for (int t = pair; ok && t < tiles; t += npairs) {
                 int g, lt;
                 locate(t, g, lt);
                 const Params& p = args.p[g];
-                if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) break;
+                const int kst = p.ks_total;
+                if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY) ||
+                    !wait_fast(B_FULL(stage), phase, abort_flag, ERR_FULL)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
-                for (int ks = 0; ks < p.ks_total; ++ks) {
-                    if (!wait_fast(B_FULL(stage), phase, abort_flag, ERR_FULL) ||
-                        !wait_fast(B_SFREADY(stage), phase, abort_flag, ERR_FULL)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                for (int ks = 0; ks < kst; ++ks) {
+                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
                     const uint64_t ad = adesc0 + (uint64_t)(stage * kDescPerStage);
                     const uint64_t bd = bdesc0 + (uint64_t)(stage * kDescPerStage);
                     const uint32_t tsf = tsf0 + stage * C::SF_COLS;
-                    const uint32_t tsfb = tsf + C::SFA_COLS;
-                    const uint32_t acc0 = ks > 0 ? 1u : 0u;
-                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
-                    if (nk == 4) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int chunk = MX ? (j >> 1) : j;
-                            tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
-                                            (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
-                                            tsfb + chunk * 8, j > 0 ? 1u : acc0);
-                        }
-                    } else {
-                        for (int j = 0; j < nk; ++j) {
-                            const int chunk = MX ? (j >> 1) : j;
-                            tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
-                                            (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
-                                            tsfb + chunk * 8, j > 0 ? 1u : acc0);
-                        }
+                    auto mma = [&](int j) {
+                        const int chunk = MX ? (j >> 1) : j;
+                        tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j, (MX && (j & 1)) ? idesc2 : idesc0,
+                                        tsf + 4 * chunk, tsf + C::SFA_COLS + chunk * 8,
+                                        (j > 0 || ks > 0) ? 1u : 0u);
+                    };
+                    mma(0);
+                    if (pending >= 0) tc_commit_pair_both(B_EMPTY(pending));
+                    if (nk > 1) mma(1);
+                    int nstage = stage + 1;
+                    uint32_t nphase = phase;
+                    if (nstage == STAGES) {
+                        nstage = 0;
+                        nphase ^= 1u;
                     }
-                    tc_commit_pair_both(B_EMPTY(stage));
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    const bool more = ks + 1 < kst;
+                    const bool ready = more && mbar_test_wait(B_FULL(nstage), nphase);
+                    if (nk > 2) mma(2);
+                    if (nk > 3) mma(3);
+                    pending = stage;
+                    stage = nstage;
+                    phase = nphase;
+                    if (more) {
+                        if (!ready && !wait_bounded(B_FULL(stage), phase, abort_flag, ERR_FULL)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
                     }
                 }
                 if (!ok) break;
+                tc_commit_pair_both(B_EMPTY(pending));
+                pending = -1;
                 tc_commit_pair_both(acc_full);
                 acc_phase ^= 1u;
             }
+            if (pending >= 0) tc_commit_pair_both(B_EMPTY(pending));
             // every pair MMA issued here has completed before the TMEM is freed
             asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                              drain)
                          : "memory");
             wait_drain(drain, 0);
         }
-    } else if (warp < 6) {
-        // ---------------- epilogue (warps 2..5, both CTAs) ----------------
-        const int q = warp & 3;
-        const int row = q * 32 + lane;
+        __syncwarp();
+    } else if (warp < 6 || warp >= 10) {
+        // ---------------- epilogue (warps 2..5 and 10..13, both CTAs) ----------------
+        const int q = warp & 3;                      // TMEM lane quadrant
+        const int half = warp >= 10 ? 1 : 0;         // accumulator columns [128 half, 128 half + 128)
+        const int eb = half * 4 + q;                 // staging block
         pdl_wait();
-        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16);
+        const uint32_t trow = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 128);
         const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
         for (int t = pair; t < tiles; t += npairs) {
@@ -1268,23 +1351,30 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             locate(t, g, lt);
             const Params& p = args.p[g];
             const float alpha = p.alpha ? *p.alpha : 1.0f;
-            int ok = 0;
-            if (lane == 0) ok = wait_bounded(acc_full, acc_phase, abort_flag, ERR_ACC_FULL) ? 1 : 0;
-            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-            if (!ok) break;
-            __syncwarp();
+            if (!warp_wait(acc_full, acc_phase, abort_flag, ERR_ACC_FULL)) break;
             tc_fence_after();
-            uint32_t packed[PAIR_BN / 2];
-#pragma unroll
-            for (int c = 0; c < PAIR_BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(trow + c * 32, r);
-                tmem_wait_ld(r);
+            // four 32-column loads, two buffers: each load overlaps the
+            // conversion of the previous chunk
+            uint32_t packed[64];
+            uint32_t ra[32], rb[32];
+            auto convert = [&](const uint32_t (&r)[32], int c) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
                     packed[c * 16 + i] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[2 * i])),
                                                      __fmul_rn(alpha, __uint_as_float(r[2 * i + 1])));
-            }
+            };
+            tmem_ld32(trow, ra);
+            tmem_wait_ld(ra);
+            tmem_ld32(trow + 32, rb);
+            convert(ra, 0);
+            tmem_wait_ld(rb);
+            tmem_ld32(trow + 64, ra);
+            convert(rb, 1);
+            tmem_wait_ld(ra);
+            tmem_ld32(trow + 96, rb);
+            convert(ra, 2);
+            tmem_wait_ld(rb);
+            convert(rb, 3);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -1299,13 +1389,13 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             // one lane stores the block with TMA, coalesced and clipped to D.
             const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
             const int y0 = (tm * 2 + (int)rank) * BM + q * 32;
-            const uint32_t blk = smem0 + C::OFF_EPI + q * C::EPI_BLOCK;
+            const uint32_t blk = smem0 + C::OFF_EPI + eb * C::EPI_BLOCK;
             const uint32_t my_row = blk + lane * 64;
             const int sw = (lane >> 1) & 3;
             if (y0 < p.rows_a) {
 #pragma unroll
-                for (int c = 0; c < PAIR_BN / 32; ++c) {
-                    const int x0 = tn * PAIR_BN + c * 32;
+                for (int c = 0; c < 4; ++c) {
+                    const int x0 = tn * PAIR_BN + half * 128 + c * 32;
                     if (x0 >= p.rows_b) break;
                     if (lane == 0) bulk_wait_read_all();   // the block's previous store has read it
                     __syncwarp();
@@ -1323,9 +1413,11 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             acc_phase ^= 1u;
         }
         if (lane == 0) bulk_wait_all();   // every store of D has completed
+        __syncwarp();
     } else {
         // ---------------- scale staging (warps 6..9, both CTAs) ----------------
         const uint32_t tq = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t full_leader0 = map_to_rank(B_FULL(0), 0);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -1339,14 +1431,10 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             for (int h = 0; h < 2; ++h)
                 if (tn * 2 + h < p.sfb_row_tiles) ++nbh;
             for (int ks = 0; ks < p.ks_total; ++ks) {
-                int w = 0;
-                if (lane == 0) w = wait_fast(B_SFFULL(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
-                w = __shfl_sync(0xFFFFFFFFu, w, 0);
-                if (!w) {
+                if (!warp_wait(B_SFFULL(stage), phase, abort_flag, ERR_FULL)) {
                     ok = false;
                     break;
                 }
-                __syncwarp();
                 tc_fence_after();
                 const int nk = min(4, (p.K - ks * BK) / MMA_K);
                 const int nch = MX ? nk / 2 : nk;
@@ -1387,10 +1475,11 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
                 __syncwarp();
                 if (lane == 0) {
                     if (leader)
-                        mbar_arrive(B_SFREADY(stage));
+                        mbar_arrive(B_FULL(stage));
                     else
-                        mbar_arrive_cluster_relaxed(map_to_rank(B_SFREADY(stage), 0));
+                        mbar_arrive_cluster_relaxed(full_leader0 + 8u * stage);
                 }
+                __syncwarp();
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -1635,7 +1724,7 @@ cudaError_t launch_pair_kernel(const PairArgs<NG>& args, int grid, cudaStream_t 
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kPairThreads, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
@@ -1653,7 +1742,7 @@ cudaError_t launch_pair_kernel(const PairArgs<NG>& args, int grid, cudaStream_t 
 }
 
 constexpr int PAIR_STAGES_NV = 5;   // 38 KB per stage
-constexpr int PAIR_STAGES_MX = 6;   // 35 KB per stage
+constexpr int PAIR_STAGES_MX = 5;   // 35 KB per stage
 
 // Fills problem slot g of a pair-kernel launch (tensor maps and Params).
 template <int NG>
