@@ -589,6 +589,63 @@ class PrefillWorkload(Workload):
                 "sample": self.sample_note(tiles) + "; %.1f s of CPU work in the measured sample" % spent}
 
 
+class TorchCall:
+    """A comparison-point call into a library (torch) inside a step; it runs
+    on the current stream, so on_stream only records nothing new."""
+
+    def __init__(self, fn, name):
+        self.fn, self.name = fn, name
+
+    def __call__(self):
+        self.fn()
+
+    def on_stream(self, stream):
+        return self
+
+
+class W4A16Workload(Workload):
+    """The W4A16 comparison path: per step the NVFP4 weights are
+    reconstructed to BF16 (this library's fp4_dequantize) and a 16-bit GEMM
+    (torch.matmul, i.e. cuBLAS) multiplies the BF16 activation by them.  A
+    comparison point for the native W4A4 path on the same shapes, not part
+    of the product."""
+
+    def __init__(self, M, N, K, dev, stream=None, act=None):
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.M, self.N, self.K = M, N, K
+        self.name = "W4A16 comparison: NVFP4 weights -> BF16, then BF16 GEMM, M=%d N=%d K=%d" % (M, N, K)
+        if M <= 16:
+            W = synth.decode_weight(N, K)
+            A = synth.decode_activation(M, K)
+        else:
+            A, W = synth.prefill(M, N, K)
+        Wd = _dev_bf16(W, dev)
+        gW = fp4.global_scale(Wd)
+        pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
+        del Wd
+        Ad = _dev_bf16(A, dev)
+        W16 = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        deq = fp4.BoundCall("fp4_dequantize", fp4.NVFP4, fp4._dptr(pW, "packed"), fp4._dptr(sW, "scales"),
+                            fp4._dptr(gW, "gs"), N, K, fp4._dptr(W16, "out"), K, fp4._stream(stream))
+        mm = TorchCall(lambda: torch.matmul(Ad, W16.t(), out=D), "bf16_gemm")
+        self.calls = [[[deq], [mm]]]
+        self.bufs = [(pW, sW, gW, Ad, W16, D)]
+        torch.cuda.empty_cache()
+        self.kernels = ["dequantize", "bf16_gemm"]
+        self.flops = 2.0 * M * N * K
+        self.work = {"dequantize": N * K // 2 + fp4.fp4_scale_bytes(fp4.NVFP4, N, K) + N * K * 2,
+                     "bf16_gemm": self.flops}
+        self.bound = {"dequantize": "hbm", "bf16_gemm": "tensor"}
+        self.tensor_ratio = {"bf16_gemm": 1.0}   # a BF16 contraction: the BF16 peak
+        self.launches_per_step = 1              # this library's kernels (the GEMM is cuBLAS)
+        self.dominant = "bf16_gemm"
+        self.l2_note = "BF16 weights %.0f MB > %d MB L2" % (N * K * 2 / 1e6, L2_BYTES >> 20)
+
+    def value(self, sec_per_step):
+        return self.flops / sec_per_step / 1e12
+
+
 def make_workload(name, dev, stream):
     if name == "square_mx":
         return SquareWorkload(fp4.MXFP4, 4096, dev, stream=stream)
@@ -604,6 +661,10 @@ def make_workload(name, dev, stream):
         return MoeWorkload(dev, grouped=name == "moe_grouped_mx", stream=stream)
     if name == "dequant_w_nv":
         return DequantWorkload(dev, stream=stream)
+    if name == "w4a16_prefill_up":
+        return W4A16Workload(8192, 28672, 8192, dev, stream=stream)
+    if name == "w4a16_decode_m16":
+        return W4A16Workload(16, 28672, 8192, dev, stream=stream)
     if name.startswith("quant_"):
         _, shape, f, ax = name.split("_")
         rows, cols = (16384, 16384) if shape == "16384" else (8192, 28672)
@@ -613,7 +674,7 @@ def make_workload(name, dev, stream):
 
 
 WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
-             "prefill_down", "moe_grouped_mx", "moe_separate_mx", "dequant_w_nv"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
+             "prefill_down", "moe_grouped_mx", "moe_separate_mx", "dequant_w_nv", "w4a16_prefill_up", "w4a16_decode_m16"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
                                 for f in ("nv", "mx", "p1e8") for a in ("row", "col")]
 
 
@@ -811,8 +872,9 @@ def main():
         dur = kern_ms[k] / 1e3
         if wl.bound[k] == "tensor":
             ach = wl.work[k] / dur / 1e12
-            rooflines[k] = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s",
-                            "frac": ach / fp4_peak, "ms": kern_ms[k], "in_step_ms": in_step_ms[k]}
+            peak = peaks["bf16_tflops"] * getattr(wl, "tensor_ratio", {}).get(k, FP4_PER_BF16)
+            rooflines[k] = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                            "frac": ach / peak, "ms": kern_ms[k], "in_step_ms": in_step_ms[k]}
         else:
             ach = wl.work[k] / dur / 1e9
             rooflines[k] = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -823,9 +885,10 @@ def main():
     dom["timing"] = "kernel alone, %d back-to-back launches in a graph, CUDA events" % G
     dom["traffic"] = recorded_traffic(args.workload, wl.dominant)
     dom["kernel"] = wl.dominant
+    ratio = getattr(wl, "tensor_ratio", {}).get(wl.dominant, FP4_PER_BF16)
     dom["peak_source"] = ("%s: %s" % (peaks["source"],
-                                      "bf16 burst x %.0f (nominal FP4:BF16)" % FP4_PER_BF16
-                                      if dom["bound"] == "tensor" else "HBM copy"))
+                                      ("bf16 burst x %.0f (nominal FP4:BF16)" % ratio if ratio != 1.0
+                                       else "bf16 burst") if dom["bound"] == "tensor" else "HBM copy"))
 
     e2e = None
     if not args.no_e2e and hasattr(wl, "e2e_setup"):

@@ -36,6 +36,22 @@ cudaError_t device_info(DeviceInfo* out)
 
 thread_local char g_last_error[256] = "";
 
+cudaError_t current_context(void** ctx)
+{
+    using GetCurrentFn = int (*)(void**);   // cuCtxGetCurrent, reached through the runtime
+    static GetCurrentFn fn = []() -> GetCurrentFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<GetCurrentFn>(p);
+    }();
+    if (!fn) return cudaErrorNotSupported;
+    *ctx = nullptr;
+    return fn(ctx) == 0 ? cudaSuccess : cudaErrorInvalidResourceHandle;
+}
+
 void set_last_error(const char* what, cudaError_t e)
 {
     snprintf(g_last_error, sizeof g_last_error, "%s: %s", what,
@@ -48,9 +64,9 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Formats of the GEMM entry points, and the quantizer's (which adds P1E8).
-bool valid_fmt(fp4_format f) { return f == FP4_NVFP4 || f == FP4_MXFP4; }
-bool valid_quant_fmt(fp4_format f) { return valid_fmt(f) || f == FP4_P1E8; }
+// Formats of the GEMM and quantizer entry points.
+bool valid_fmt(fp4_format f) { return f == FP4_NVFP4 || f == FP4_MXFP4 || f == FP4_P1E8; }
+bool valid_quant_fmt(fp4_format f) { return valid_fmt(f); }
 
 fp4_status from_cuda(cudaError_t e)
 {
@@ -301,7 +317,7 @@ static fp4_status validate_gemm(fp4_format fmt, const void* A, const void* sA, c
 {
     if (M < 0 || N < 0 || K < 0 || ldd < N) return FP4_ERR_INVALID_ARG;
     if (!D) return FP4_ERR_INVALID_ARG;
-    const int kq = fmt == FP4_NVFP4 ? 64 : 128;
+    const int kq = fmt == FP4_MXFP4 ? 128 : 64;   // four blocks: whole scale tiles
     if (K % kq != 0 || N % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (M >= kMaxRows || N >= kMaxRows || K / 2 >= kMaxRows) return FP4_ERR_UNSUPPORTED_SHAPE;
     if (ldd % 8 != 0 || !aligned16(D)) return FP4_ERR_MISALIGNED;
@@ -480,7 +496,7 @@ fp4_status fp4_get_device_status(fp4_stream_t stream)
     e = fp4::read_and_clear_error_word(&word);
     if (e != cudaSuccess) return from_cuda(e);
     if (!word) return FP4_OK;
-    e = fp4::clear_noalloc_counters();
+    e = fp4::clear_noalloc_counters(reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return from_cuda(e);
     return (word & fp4::kErrorWorkspaceBit) && !(word & ~fp4::kErrorWorkspaceBit) ? FP4_ERR_WORKSPACE
                                                                                      : FP4_ERR_TIMEOUT;

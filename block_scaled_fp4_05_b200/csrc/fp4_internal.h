@@ -74,8 +74,11 @@ cudaError_t launch_wait_selftest(cudaStream_t s);
 size_t noalloc_scratch_bytes();
 cudaError_t noalloc_scratch(void** out);
 // Zeroes the decode counters of the static scratch (current device), after an
-// error left them in an unknown state.
-cudaError_t clear_noalloc_counters();
+// error left them in an unknown state: a memset on stream s, then a wait for s.
+cudaError_t clear_noalloc_counters(cudaStream_t s);
+// The calling thread's current CUDA context (driver handle, as an opaque
+// pointer), for caches of per-context device addresses.
+cudaError_t current_context(void** ctx);
 // Bit of the device error word set by a decode call whose workspace counters
 // were out of range (not zeroed).
 constexpr unsigned int kErrorWorkspaceBit = 64u;

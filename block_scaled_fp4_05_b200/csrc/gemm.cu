@@ -297,13 +297,14 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
 }
 
 // Instruction descriptor of kind::mxf4nvf4 with block scaling: E2M1 x E2M1,
-// FP32 accumulate, K-major A and B, M = 128, N = BN; scale type UE8M0 (MX) or
-// UE4M3 (NV); sf_id selects the scale byte pair (2X) inside each column.
-template <int BN, bool MX>
+// FP32 accumulate, K-major A and B, M = 128, N = BN; scale type UE8M0
+// (MXFP4, and 16-element blocks with E8M0 scales) or UE4M3 (NVFP4); sf_id
+// selects the scale byte pair (2X) inside each column.
+template <int BN, int FMT>
 __device__ __forceinline__ uint32_t make_idesc(uint32_t sf_id)
 {
     return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-           ((MX ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24) | (sf_id << 29);
+           ((FMT != kNv ? 1u : 0u) << 23) | ((uint32_t)(BM >> 4) << 24) | (sf_id << 29);
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
@@ -471,11 +472,12 @@ struct Schedule {
 // ------------------------------------------------------------------------
 // The kernel
 // ------------------------------------------------------------------------
-template <int BN, int STAGES, bool MX, bool STREAM_K>
+template <int BN, int STAGES, int FMT, bool STREAM_K>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p)
 {
+    constexpr bool MX = FMT == kMx;   // 32-element blocks (scale_vec::2X); else 16 (4X)
     using C = Cfg<BN, STAGES>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -626,8 +628,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const uint64_t adesc0 = desc_sw128(smem0);
             const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
             constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;   // start-address field step
-            const uint32_t idesc0 = make_idesc<BN, MX>(0);
-            const uint32_t idesc2 = make_idesc<BN, MX>(2);
+            const uint32_t idesc0 = make_idesc<BN, FMT>(0);
+            const uint32_t idesc2 = make_idesc<BN, FMT>(2);
             const uint32_t tsf0 = tmem_base + C::SF_COL0;
             Schedule<STREAM_K> sched(p);
             Seg sg;
@@ -752,14 +754,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 // FP32 partial of this segment; the CTA whose partial completes
                 // a weight tile (per 32-row lane quadrant) sums all partials of
-                // that tile in CTA order and writes the BF16 outputs.  Ordering:
-                // the lanes' partial stores, a warp barrier, then lane 0's
-                // release-acquire increment; the last arriver's lanes read the
-                // other partials after another warp barrier.
+                // that tile in CTA order and writes the BF16 outputs.  Ordering
+                // (the usual semaphore pattern): every lane's partial stores,
+                // a device-scope fence by every lane, a warp barrier, then lane
+                // 0's release-acquire increment; in the last arriver, lane 0's
+                // acquire, a warp barrier and a fence by every lane before the
+                // other partials are read.
                 float* slot = p.ws + ((int64_t)blockIdx.x * p.max_seg + sg.slot) * (BN * BM);
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
                     if (j < p.rows_b) __stcg(slot + j * BM + row, __uint_as_float(r[j]));
+                __threadfence();
                 __syncwarp();
                 const int64_t G = gridDim.x;
                 const int64_t x0 = (int64_t)sg.tm * p.ks_total, x1 = x0 + p.ks_total - 1;
@@ -775,6 +780,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 last = __shfl_sync(0xFFFFFFFFu, last, 0);
                 if (last) {
                     __syncwarp();
+                    __threadfence();
                     const int64_t n = (int64_t)sg.tm * BM + row;
                     float sum[16];
 #pragma unroll
@@ -1070,11 +1076,11 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
 }
 
 // Instruction descriptor of the pair MMA: M = 256 (128 rows per CTA), N = 256.
-template <bool MX>
+template <int FMT>
 __device__ __forceinline__ uint32_t make_idesc_pair(uint32_t sf_id)
 {
     return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PAIR_BN >> 3) << 17) |
-           ((MX ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
+           ((FMT != kNv ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
 }
 
 __device__ __forceinline__ void spin_ns(uint64_t ns)
@@ -1131,10 +1137,11 @@ struct PairArgs {
     int tile_begin[NG + 1];
 };
 
-template <int STAGES, bool MX, int NG>
+template <int STAGES, int FMT, int NG>
 __global__ void __launch_bounds__(kPairThreads, 1)
 fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
 {
+    constexpr bool MX = FMT == kMx;   // 32-element blocks (scale_vec::2X); else 16 (4X)
     using C = PairCfg<STAGES, MX>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -1270,8 +1277,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             const uint64_t adesc0 = desc_sw128(smem0);
             const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
             constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;
-            const uint32_t idesc0 = make_idesc_pair<MX>(0);
-            const uint32_t idesc2 = make_idesc_pair<MX>(2);
+            const uint32_t idesc0 = make_idesc_pair<FMT>(0);
+            const uint32_t idesc2 = make_idesc_pair<FMT>(2);
             const uint32_t tsf0 = tmem_base + C::SF_COL0;
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
@@ -1562,7 +1569,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes,
 
 // Raises the kernel's dynamic shared-memory limit once per device; the
 // statics are distinct for every instantiation of the kernel template.
-template <int BN, int STAGES, bool MX, bool STREAM_K>
+template <int BN, int STAGES, int FMT, bool STREAM_K>
 cudaError_t set_smem_once(int bytes)
 {
     static std::mutex mu;
@@ -1572,18 +1579,18 @@ cudaError_t set_smem_once(int bytes)
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     if (dev < 64 && ((done_mask >> dev) & 1ull)) return cudaSuccess;
-    e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>,
+    e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, STAGES, FMT, STREAM_K>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess && dev < 64) done_mask |= 1ull << dev;
     return e;
 }
 
-template <int BN, int STAGES, bool MX, bool STREAM_K>
+template <int BN, int STAGES, int FMT, bool STREAM_K>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p, int grid,
                           cudaStream_t s)
 {
     using C = Cfg<BN, STAGES>;
-    cudaError_t e = set_smem_once<BN, STAGES, MX, STREAM_K>(C::SMEM);
+    cudaError_t e = set_smem_once<BN, STAGES, FMT, STREAM_K>(C::SMEM);
     if (e != cudaSuccess) {
         set_last_error("cudaFuncSetAttribute(max dynamic shared memory)", e);
         return e;
@@ -1598,10 +1605,10 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>, ta, tb, p);
+    e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, STAGES, FMT, STREAM_K>, ta, tb, p);
     if (e != cudaSuccess) {
         cudaFuncAttributes fa{};
-        cudaFuncGetAttributes(&fa, fp4_gemm_kernel<BN, STAGES, MX, STREAM_K>);
+        cudaFuncGetAttributes(&fa, fp4_gemm_kernel<BN, STAGES, FMT, STREAM_K>);
         int dev = 0, optin = 0;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
@@ -1701,11 +1708,11 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.max_seg = 0;
 }
 
-template <int STAGES, bool MX, int NG>
+template <int STAGES, int FMT, int NG>
 cudaError_t launch_pair_kernel(const PairArgs<NG>& args, int grid, cudaStream_t s)
 {
-    using C = PairCfg<STAGES, MX>;
-    auto kern = fp4_gemm_pair_kernel<STAGES, MX, NG>;
+    using C = PairCfg<STAGES, FMT == kMx>;
+    auto kern = fp4_gemm_pair_kernel<STAGES, FMT, NG>;
     static std::mutex mu;
     static uint64_t done_mask = 0;
     int dev = 0;
@@ -1766,8 +1773,9 @@ cudaError_t launch_pair(const PairArgs<NG>& args, int fmt, const DeviceInfo& dev
     if (tiles == 0) return cudaSuccess;
     const int64_t max_pairs = dev.sm_count / 2;
     const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
-    if (fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, true, NG>(args, grid, s);
-    return launch_pair_kernel<PAIR_STAGES_NV, false, NG>(args, grid, s);
+    if (fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, kMx, NG>(args, grid, s);
+    if (fmt == kP1) return launch_pair_kernel<PAIR_STAGES_NV, kP1, NG>(args, grid, s);
+    return launch_pair_kernel<PAIR_STAGES_NV, kNv, NG>(args, grid, s);
 }
 
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s)
@@ -1829,8 +1837,9 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     p.counters = static_cast<int*>(a.ws);
     p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(a.ws) + kDecodeCounterBytes);
     if (a.fmt == kMx)
-        return launch_kernel<DECODE_BN, DECODE_STAGES, true, true>(tw, tx, p, G, s);
-    return launch_kernel<DECODE_BN, DECODE_STAGES, false, true>(tw, tx, p, G, s);
+        return launch_kernel<DECODE_BN, DECODE_STAGES, kMx, true>(tw, tx, p, G, s);
+    if (a.fmt == kP1) return launch_kernel<DECODE_BN, DECODE_STAGES, kP1, true>(tw, tx, p, G, s);
+    return launch_kernel<DECODE_BN, DECODE_STAGES, kNv, true>(tw, tx, p, G, s);
 }
 
 // ------------------------------------------------------------------------
@@ -1846,37 +1855,46 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchB
 
 size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
-// Device address of g_decode_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with that device current and cached.
+// Device address of g_decode_scratch in the current context.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device with that device current and cached together with the
+// context it belongs to; a new context on the device (e.g. after
+// cudaDeviceReset) makes the lookup run again.
 cudaError_t noalloc_scratch(void** out)
 {
     static std::mutex mu;
     static void* cache[64] = {};
+    static void* cache_ctx[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    void* ctx = nullptr;
+    e = current_context(&ctx);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    if (dev < 64 && cache[dev]) {
+    if (dev < 64 && cache[dev] && cache_ctx[dev] == ctx) {
         *out = cache[dev];
         return cudaSuccess;
     }
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 64) cache[dev] = ptr;
+    if (dev < 64) {
+        cache[dev] = ptr;
+        cache_ctx[dev] = ctx;
+    }
     *out = ptr;
     return cudaSuccess;
 }
 
-cudaError_t clear_noalloc_counters()
+cudaError_t clear_noalloc_counters(cudaStream_t s)
 {
     void* ptr = nullptr;
     cudaError_t e = noalloc_scratch(&ptr);
     if (e != cudaSuccess) return e;
-    e = cudaMemset(ptr, 0, kDecodeCounterBytes);
+    e = cudaMemsetAsync(ptr, 0, kDecodeCounterBytes, s);
     if (e != cudaSuccess) return e;
-    return cudaDeviceSynchronize();
+    return cudaStreamSynchronize(s);
 }
 
 cudaError_t launch_wait_selftest(cudaStream_t s)

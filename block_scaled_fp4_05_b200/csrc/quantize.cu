@@ -243,9 +243,14 @@ quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
 // Dequantization (reconstruction) x_hat = q * S_block (* S_global) of a
 // rowwise-quantized operand [rows x k] into BF16, rounded once to nearest
 // even: the product of the E2M1 value, the block scale and S_global is exact
-// in FP64 (at most 2 + 4 + 24 significant bits), then converted.  Thread t
-// takes 16 packed bytes (32 codes) of one row; HBM-bound (0.5 + 1/blk bytes
-// read, 2 written per element).
+// in FP64 (at most 2 + 4 + 24 significant bits), then converted.  HBM-bound
+// (0.5 + 1/blk bytes read, 2 written per element).
+// A warp takes 1024 consecutive codes of one row (4 segments of 256): in each
+// segment lane l owns codes [8l, 8l + 8), one 4-byte load of packed codes and
+// one 16-byte store of BF16, so every warp load covers 128 contiguous bytes
+// and every warp store 512.  The 8 magnitudes of a block's scale (the
+// rounding table) are computed by two neighbouring lanes, four each, and
+// exchanged with shuffles.
 // ---------------------------------------------------------------------------
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
@@ -255,55 +260,76 @@ dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict_
 {
     pdl_trigger();
     constexpr int KB = FMT == kMx ? 32 : 16;
+    constexpr int SEG = 256;                            // codes per warp segment
+    constexpr int UNROLL = 4;
     const double gs = FMT != kMx ? (double)__ldg(gs_ptr) : 1.0;
-    const int64_t cpr = k / 32;                         // 16-byte packed chunks per row
+    const int lane = threadIdx.x & 31;
     const int64_t nsc = k / KB;                         // scales per row
     const int64_t nct = (nsc + 3) / 4;                  // scale tiles per 128-row group
-    const int64_t total = rows * cpr;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < total;
-         u += (int64_t)gridDim.x * kThreads) {
-        const int64_t r = u / cpr, c = u - r * cpr;
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(packed + r * (k / 2)) + c);
-        const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-        uint32_t o[16];
+    const int64_t groups_per_row = (k + SEG * UNROLL - 1) / (SEG * UNROLL);
+    const int64_t total = rows * groups_per_row;
+    const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
+    const int half = lane & 1;                          // which four table entries this lane forms
+    for (int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < total; w += warps) {
+        const int64_t r = w / groups_per_row;
+        const int64_t c_base = (w - r * groups_per_row) * (SEG * UNROLL);
+        const uint8_t* prow = packed + r * (k / 2);
+        const uint8_t* srow = scales + (r / 128) * nct * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4;
+        uint32_t words[UNROLL];
+        uint8_t sbytes[UNROLL];
 #pragma unroll
-        for (int b = 0; b < 32 / KB; ++b) {
-            const int64_t blk = c * (32 / KB) + b;      // block index within the row
-            const uint8_t sb = __ldg(scales + ((r / 128) * nct + blk / 4) * 512 + (r % 32) * 16 +
-                                     ((r / 32) % 4) * 4 + blk % 4);
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t c0 = c_base + u * SEG + lane * 8;    // first code of this lane
+            const bool in = c0 < k;
+            words[u] = in ? __ldg(reinterpret_cast<const uint32_t*>(prow + c0 / 2)) : 0u;
+            const int64_t blk = c0 / KB;
+            sbytes[u] = in ? __ldg(srow + (blk / 4) * 512 + blk % 4) : (uint8_t)0;
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t c0 = c_base + u * SEG + lane * 8;
             double s;
             if (FMT == kNv) {
-                s = (double)e4m3_value(sb);
+                s = (double)e4m3_value(sbytes[u]);
             } else {
-                s = __longlong_as_double((long long)(sb + 896) << 52);   // 2^(sb - 127), exact
+                s = __longlong_as_double((long long)(sbytes[u] + 896) << 52);   // 2^(byte - 127), exact
             }
             const double eff = s * gs;
-            // BF16 of the 8 magnitudes q * eff (q = 0, .5, 1, 1.5, 2, 3, 4, 6),
-            // each exact in FP64 and rounded once; the sign of a code is the
-            // BF16 sign bit (rounding to nearest even is symmetric)
-            constexpr double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
-            uint32_t t[4];
+            // this lane's four entries of the table, the neighbour's four by shuffle
+            // E2M1 magnitudes 0, .5, 1, 1.5 (even lane) or 2, 3, 4, 6 (odd lane)
+            const double q0 = half ? 2.0 : 0.0, q1 = half ? 3.0 : 0.5;
+            const double q2 = half ? 4.0 : 1.0, q3 = half ? 6.0 : 1.5;
+            uint32_t mine[2], other[2];
+            mine[0] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(q0 * eff)) |
+                      ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(q1 * eff)) << 16);
+            mine[1] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(q2 * eff)) |
+                      ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(q3 * eff)) << 16);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                t[j] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(kE2M1[2 * j] * eff)) |
-                       ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(kE2M1[2 * j + 1] * eff)) << 16);
+            for (int j = 0; j < 2; ++j) other[j] = __shfl_xor_sync(0xFFFFFFFFu, mine[j], 1);
+            // magnitudes 0..7 as BF16 pairs: t[0] = {0, 1}, t[1] = {2, 3}, ...
+            // (both lanes of a pair hold the same block: 8 codes per lane and
+            // at least 16 per block)
+            const uint32_t t0 = half ? other[0] : mine[0];
+            const uint32_t t1 = half ? other[1] : mine[1];
+            const uint32_t t2 = half ? mine[0] : other[0];
+            const uint32_t t3 = half ? mine[1] : other[1];
             auto lookup = [&](uint32_t nib) {
-                const uint32_t lo = (nib & 2u) ? t[1] : t[0];
-                const uint32_t hi = (nib & 2u) ? t[3] : t[2];
+                const uint32_t lo = (nib & 2u) ? t1 : t0;
+                const uint32_t hi = (nib & 2u) ? t3 : t2;
                 const uint32_t w2 = (nib & 4u) ? hi : lo;
                 const uint32_t mag = (nib & 1u) ? (w2 >> 16) : (w2 & 0xFFFFu);
                 return mag | ((nib & 8u) << 12);
             };
+            if (c0 < k) {
+                uint32_t o[4];
 #pragma unroll
-            for (int i = 0; i < KB / 2; ++i) {          // two codes per output word
-                const int e = b * KB + 2 * i;           // element within the 32
-                const uint32_t byte = (words[e / 8] >> ((e % 8) * 4)) & 0xFFu;
-                o[e / 2] = lookup(byte & 0xFu) | (lookup(byte >> 4) << 16);
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t byte = (words[u] >> (8 * i)) & 0xFFu;
+                    o[i] = lookup(byte & 0xFu) | (lookup(byte >> 4) << 16);
+                }
+                *reinterpret_cast<uint4*>(out + r * ld + c0) = make_uint4(o[0], o[1], o[2], o[3]);
             }
         }
-        uint4* dst = reinterpret_cast<uint4*>(out + r * ld + c * 32);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
     }
 }
 
@@ -612,22 +638,29 @@ __global__ void alpha_kernel(const float* a, const float* b, float* out)
     *out = __fmul_rn(*a, *b);
 }
 
-// Device address of the slot ring on the current device (looked up once per
-// device: in host code the array's name is not a device address).
+// Device address of the slot ring in the current context (looked up once per
+// device and context: in host code the array's name is not a device address).
 cudaError_t gs_slots(GsSlot** out)
 {
     static std::mutex mu;
     static GsSlot* cache[64] = {};
+    static void* cache_ctx[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    void* ctx = nullptr;
+    e = current_context(&ctx);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
-    if (dev < 64 && cache[dev]) {
+    if (dev < 64 && cache[dev] && cache_ctx[dev] == ctx) {
         *out = cache[dev];
         return cudaSuccess;
     }
     e = cudaGetSymbolAddress(reinterpret_cast<void**>(out), g_gs_slots);
-    if (e == cudaSuccess && dev < 64) cache[dev] = *out;
+    if (e == cudaSuccess && dev < 64) {
+        cache[dev] = *out;
+        cache_ctx[dev] = ctx;
+    }
     return e;
 }
 
@@ -786,8 +819,8 @@ cudaError_t launch_dequantize(int fmt, const uint8_t* packed, const uint8_t* sca
     DeviceInfo dev;
     cudaError_t e = device_info(&dev);
     if (e != cudaSuccess) return e;
-    const int64_t chunks = rows * (k / 32);
-    int64_t grid = (chunks + kThreads - 1) / kThreads;
+    const int64_t warps = rows * ((k + 1023) / 1024);
+    int64_t grid = (warps + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = (int64_t)dev.sm_count * 8;
     if (grid > cap) grid = cap;
     if (fmt == kNv)

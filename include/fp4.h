@@ -64,8 +64,9 @@ typedef enum {
     /* 16-element blocks with an E8M0 block scale under an FP32 S_global:
      * S_block = 2^ceil(log2(max(amax / (6 S_global), 1e-8))) (capped at
      * 2^127), the NVFP4 of [NVFP4-Arch] "1. The Dual-Level Mathematical
-     * Formulation" read literally (its block scale is E8M0).  Quantizer only:
-     * the GEMM entry points reject it. */
+     * Formulation" read literally (its block scale is E8M0).  The GEMM runs
+     * it as the 16-element block-scaled MMA with the UE8M0 scale type, with
+     * alpha = S_global,A * S_global,B as for NVFP4. */
     FP4_P1E8 = 2
 } fp4_format;
 
@@ -270,7 +271,7 @@ fp4_status fp4_alpha_from_global_scales(const float* gsA, const float* gsB, floa
  *          returns FP4_ERR_WORKSPACE; after that, or after FP4_ERR_TIMEOUT,
  *          zero the workspace again.  Two calls that run at the same time
  *          need two workspaces.
- * Requires K % 64 == 0 (NVFP4) or K % 128 == 0 (MXFP4) and N % 8 == 0.  M and
+ * Requires K % 64 == 0 (NVFP4, P1E8) or K % 128 == 0 (MXFP4) and N % 8 == 0.  M and
  * N tails are handled inside the kernels.  M == 0 or N == 0 is a no-op;
  * K == 0 writes zeros.
  *
@@ -340,7 +341,9 @@ size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K)
  *  - Every GPU that loads the library holds the 4 MiB until the process exits.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is cached per device and
+ *    context: after a cudaDeviceReset the next call looks it up again (and
+ *    should, like the first, come before any capture).
  *  - All calls share the array.  It is zero when the library loads, and its
  *    counters (see fp4_gemm's workspace) are zero again after every call
  *    that completes; fp4_get_device_status zeroes them after reporting an
@@ -363,7 +366,9 @@ fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA
  * FP4_ERR_WORKSPACE if a decode call found its workspace counters not zero
  * (outputs unspecified), else FP4_OK; FP4_ERR_CUDA if the synchronization
  * itself failed.  After an error it also zeroes the counters of the static
- * scratch of fp4_gemm_decode_noalloc.
+ * scratch of fp4_gemm_decode_noalloc (a memset on `stream`, waited for):
+ * every other stream that may hold an fp4_gemm_decode_noalloc call must be
+ * idle when this is called, or that call's counters are cleared under it.
  */
 fp4_status fp4_get_device_status(fp4_stream_t stream);
 

@@ -100,17 +100,20 @@ def test_quantize_batch_host_checks_without_gpu():
         assert call(0, [good]) == 6                                      # valid, but no device here
 
 
-def test_p1e8_is_a_quantizer_format_only(orc):
-    # 16-element blocks: the same sizes as NVFP4; S_global is required; the
-    # GEMM entry points reject the format before touching the device
+def test_p1e8_host_checks(orc):
+    # 16-element blocks: the same sizes and K rule as NVFP4; S_global is
+    # required by the quantizer; the GEMM accepts the format
+    import torch
     L = fp4.lib()
     for rows, K in [(1, 512), (129, 8192)]:
         assert fp4.fp4_scale_bytes(fp4.P1E8, rows, K) == orc.scale_bytes(rows, K // 16)
     assert L.fp4_quantize(2, 0, A16, 128, 512, 512, A16, A16, None, None) == 1
     assert L.fp4_quantize(2, 0, A16, 128, 480, 480, A16, A16, A16, None) == 2
     g = L.fp4_gemm_with_kernel
-    assert g(2, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 1
-    assert L.fp4_gemm_workspace_bytes(2, 16, 1024, 1024) == 0
+    assert g(2, A16, A16, A16, A16, 16, 16, 96, None, A16, 16, None, 0, 0, None) == 2   # K % 64
+    assert g(2, A16, A16, A16, A16, 16, 12, 64, None, A16, 16, None, 0, 0, None) == 2   # N % 8
+    if not torch.cuda.is_available():
+        assert g(2, A16, A16, A16, A16, 16, 16, 64, None, A16, 16, None, 0, 0, None) == 6
 
 
 def test_gemm_grouped_host_checks_without_gpu():
@@ -125,7 +128,6 @@ def test_gemm_grouped_host_checks_without_gpu():
     a = 1 << 20
     good = G(a, a, a, a, 16, 16, 64, None, a, 16)
     assert call(9, [good]) == 1                                         # bad format
-    assert call(2, [good]) == 1                                         # P1E8: quantizer only
     assert L.fp4_gemm_grouped(0, -1, None, None) == 1
     assert call(0, [good, G(a, a, a, a, 16, 16, 96, None, a, 16)]) == 2  # K % 64
     assert call(0, [good, G(a, a, a, a, 16, 12, 64, None, a, 16)]) == 2  # N % 8

@@ -10,12 +10,12 @@ from block_scaled_fp4_05_b200 import fp4, synth
 from gpu_util import assert_gemm_close, bf16_dev_to_f64, to_dev_bf16, to_dev_f32, to_dev_u8
 
 pytestmark = pytest.mark.gpu
-FMTS = [fp4.NVFP4, fp4.MXFP4]
+FMTS = [fp4.NVFP4, fp4.MXFP4, fp4.P1E8]   # P1E8: 16-element blocks, E8M0 scales under S_global
 
 
 def oracle_operands(orc, fmt, A_bits, B_bits):
-    gsA = orc.global_scale(A_bits) if fmt == fp4.NVFP4 else 1.0
-    gsB = orc.global_scale(B_bits) if fmt == fp4.NVFP4 else 1.0
+    gsA = orc.global_scale(A_bits) if fmt != fp4.MXFP4 else 1.0
+    gsB = orc.global_scale(B_bits) if fmt != fp4.MXFP4 else 1.0
     pA, sA = orc.quantize(fmt, 0, A_bits, gs=gsA)
     pB, sB = orc.quantize(fmt, 0, B_bits, gs=gsB)
     alpha = float(np.float32(gsA) * np.float32(gsB))
@@ -65,7 +65,7 @@ def test_tiny_config(orc, fmt):
                                  (300, 520, 1024), (128, 256, 2048), (257, 512, 128)])
 def test_prefill_ragged_shapes(orc, fmt, MNK):
     M, N, K = MNK
-    if K % (64 if fmt == fp4.NVFP4 else 128):
+    if K % (128 if fmt == fp4.MXFP4 else 64):
         pytest.skip("K not supported by the format")
     A = synth.normal_bf16(M, K, seed=31, outlier_factor=50.0)
     B = synth.normal_bf16(N, K, seed=31, tensor_id=1, sigma=0.02)
@@ -82,7 +82,7 @@ def test_prefill_ragged_shapes(orc, fmt, MNK):
                                  (16, 38400, 1024), (9, 38400, 1088)])
 def test_decode_kernel_shapes(orc, fmt, MNK):
     M, N, K = MNK
-    if K % (64 if fmt == fp4.NVFP4 else 128):
+    if K % (128 if fmt == fp4.MXFP4 else 64):
         pytest.skip("K not supported by the format")
     A = synth.normal_bf16(M, K, seed=32, outlier_factor=100.0)
     W = synth.normal_bf16(N, K, seed=32, tensor_id=1, sigma=0.02)
@@ -201,7 +201,7 @@ def test_end_to_end_gpu_quantize_then_gemm(orc, fmt):
     A = synth.normal_bf16(333, 1024, seed=33, outlier_factor=50.0)
     B = synth.normal_bf16(264, 1024, seed=33, tensor_id=1)
     Ad, Bd = to_dev_bf16(A), to_dev_bf16(B)
-    if fmt == fp4.NVFP4:
+    if fmt != fp4.MXFP4:
         gA, gB = fp4.global_scale(Ad), fp4.global_scale(Bd)
         alpha = torch.empty(1, dtype=torch.float32, device="cuda")
         fp4.fp4_alpha_from_global_scales(gA, gB, alpha)
@@ -223,10 +223,10 @@ def sampled_check(orc, fmt, A_bits, B_bits, kernel, n_pairs=4096):
     M, K = A_bits.shape
     N = B_bits.shape[0]
     Ad, Bd = to_dev_bf16(A_bits), to_dev_bf16(B_bits)
-    gsA = orc.global_scale(A_bits) if fmt == fp4.NVFP4 else 1.0
-    gsB = orc.global_scale(B_bits) if fmt == fp4.NVFP4 else 1.0
-    pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, to_dev_f32(gsA) if fmt == fp4.NVFP4 else None)
-    pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, to_dev_f32(gsB) if fmt == fp4.NVFP4 else None)
+    gsA = orc.global_scale(A_bits) if fmt != fp4.MXFP4 else 1.0
+    gsB = orc.global_scale(B_bits) if fmt != fp4.MXFP4 else 1.0
+    pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, to_dev_f32(gsA) if fmt != fp4.MXFP4 else None)
+    pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, to_dev_f32(gsB) if fmt != fp4.MXFP4 else None)
     alpha = float(np.float32(gsA) * np.float32(gsB))
     D = fp4.gemm(fmt, pA, sA, pB, sB, K, alpha=to_dev_f32(alpha), kernel=kernel)
     torch.cuda.synchronize()
@@ -274,7 +274,7 @@ def test_grouped_gemm_matches_oracle_per_problem(orc, fmt):
     shapes = [(int(m), N, K) for m in rng.integers(0, 300, 15)] + [(0, N, K), (40, 264, 640), (5, 136, 0)]
     items, checks = [], []
     for i, (M, Ni, Ki) in enumerate(shapes):
-        if Ki and Ki % (64 if fmt == fp4.NVFP4 else 128):
+        if Ki and Ki % (128 if fmt == fp4.MXFP4 else 64):
             Ki = 768
         Ms = max(M, 1)
         A = synth.normal_bf16(Ms, max(Ki, 128), seed=37 + i, outlier_factor=50.0)[:M, :Ki]

@@ -5,9 +5,9 @@ FP4_GEMM_DECODE), through the C ABI.
 The no-alloc form exists for callers that cannot allocate device memory on
 their hot path (a plug-in inside a framework that owns the GPU's memory pool,
 or a latency-bound loop where cudaMalloc would synchronize the device); its
-split-K partials live in a fixed array inside the library.  Two calls in a
-row on different shapes check that the second call does not depend on what
-the first one left in that shared array.
+split-K partials live in a fixed array inside the library.  Calls in a row
+on different shapes and formats check each result against the oracle and
+that no call depends on what the previous one left in that shared array.
 
 Kept in a file that sorts last, so that a run stopping at the first failure
 has already run every other test."""
@@ -35,38 +35,48 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else None
 
 
-def _operands(M, N, K, seed):
+def _operands(fmt, M, N, K, seed):
     A = synth.normal_bf16(M, K, seed=seed, outlier_factor=100.0)
     W = synth.normal_bf16(N, K, seed=seed, tensor_id=1, sigma=0.02)
     Ad = synth.bits_to_torch(A).cuda()
     Wd = synth.bits_to_torch(W).cuda()
-    gA, gW = fp4.global_scale(Ad), fp4.global_scale(Wd)
-    alpha = torch.empty(1, dtype=torch.float32, device="cuda")
-    fp4.fp4_alpha_from_global_scales(gA, gW, alpha)
-    pA, sA = fp4.quantize(Ad, fp4.NVFP4, fp4.ROWWISE, gA)
-    pW, sW = fp4.quantize(Wd, fp4.NVFP4, fp4.ROWWISE, gW)
+    if fmt == fp4.NVFP4:
+        gA, gW = fp4.global_scale(Ad), fp4.global_scale(Wd)
+        alpha = torch.empty(1, dtype=torch.float32, device="cuda")
+        fp4.fp4_alpha_from_global_scales(gA, gW, alpha)
+    else:
+        gA = gW = alpha = None
+    pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, gA)
+    pW, sW = fp4.quantize(Wd, fmt, fp4.ROWWISE, gW)
     return (A, W, gA, gW), (pA, sA, pW, sW, alpha)
 
 
-def test_noalloc_decode_matches_workspace_decode_on_two_calls(orc):
+def test_noalloc_decode_matches_oracle_and_workspace_decode_on_two_calls(orc):
+    # three calls in a row on different shapes and both formats: the shared
+    # scratch keeps what the previous call left there, and each result must
+    # still match the oracle (within the GEMM tolerance) and the workspace
+    # form of the same kernel bit for bit
     f = _noalloc()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    for M, N, K, seed in [(16, 2048, 4096, 51), (3, 1152, 2048, 52)]:
-        host, (pA, sA, pW, sW, alpha) = _operands(M, N, K, seed)
-        D_ref = fp4.gemm(fp4.NVFP4, pA, sA, pW, sW, K, alpha=alpha, kernel=fp4.GEMM_DECODE)
+    for fmt, M, N, K, seed in [(fp4.NVFP4, 16, 2048, 4096, 51), (fp4.NVFP4, 3, 1152, 2048, 52),
+                               (fp4.MXFP4, 4, 1536, 4096, 53)]:
+        host, (pA, sA, pW, sW, alpha) = _operands(fmt, M, N, K, seed)
+        D_ref = fp4.gemm(fmt, pA, sA, pW, sW, K, alpha=alpha, kernel=fp4.GEMM_DECODE)
         D_new = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-        st = f(fp4.NVFP4, _p(pA), _p(sA), _p(pW), _p(sW), M, N, K, _p(alpha), _p(D_new), N, stream)
+        st = f(fmt, _p(pA), _p(sA), _p(pW), _p(sW), M, N, K, _p(alpha), _p(D_new), N, stream)
         assert st == 0, fp4.lib().fp4_last_error()
         torch.cuda.synchronize()
         assert fp4.fp4_get_device_status() == 0
         d_ref, d_new = bf16_dev_to_f64(D_ref), bf16_dev_to_f64(D_new)
-        # tolerance of the GEMM parity tests, with S from the oracle
+        # the oracle's product of its own quantization of the same inputs
         A, W, gA, gW = host
-        gsA, gsW = np.float32(gA.item()), np.float32(gW.item())
-        qA, qsA = orc.quantize(orc.NVFP4, orc.ROWWISE, A, gs=float(gsA))
-        qW, qsW = orc.quantize(orc.NVFP4, orc.ROWWISE, W, gs=float(gsW))
-        _, S = orc.gemm(orc.NVFP4, qA, qsA, qW, qsW, alpha=float(gsA * gsW))
-        assert_gemm_close(d_new, d_ref, S, "no-alloc vs workspace decode")
+        gsA = float(np.float32(gA.item())) if gA is not None else 1.0
+        gsW = float(np.float32(gW.item())) if gW is not None else 1.0
+        ofmt = orc.NVFP4 if fmt == fp4.NVFP4 else orc.MXFP4
+        qA, qsA = orc.quantize(ofmt, orc.ROWWISE, A, gs=gsA)
+        qW, qsW = orc.quantize(ofmt, orc.ROWWISE, W, gs=gsW)
+        D_orc, S = orc.gemm(ofmt, qA, qsA, qW, qsW, alpha=float(np.float32(gsA) * np.float32(gsW)))
+        assert_gemm_close(d_new, D_orc, S, "no-alloc decode vs oracle")
         # same kernels, fixed reduction order: identical bits
         assert np.array_equal(d_new, d_ref)
 
