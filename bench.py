@@ -296,13 +296,15 @@ class SquareWorkload(Workload):
 class DecodeWorkload(Workload):
     """NVFP4 decode: W [28672 x 8192] quantized once; per step the M-token
     activation gets S_global, is quantized, and D = A_hat W_hat^T runs on the
-    swap-AB stream-K kernel."""
+    swap-AB stream-K kernel.  dynamic=True: one call, the S_global/alpha
+    launch and the decode GEMM that quantizes the activation itself."""
     unit = "GB/s"
 
-    def __init__(self, M, dev, sets=3, N=28672, K=8192, stream=None):
+    def __init__(self, M, dev, sets=3, N=28672, K=8192, stream=None, dynamic=False):
         self.stream = stream if stream is not None else torch.cuda.current_stream()
         self.M, self.N, self.K = M, N, K
-        self.name = "NVFP4 decode GEMM M=%d N=%d K=%d (W pre-quantized)" % (M, N, K)
+        self.name = "NVFP4 decode GEMM M=%d N=%d K=%d (W pre-quantized%s)" % (
+            M, N, K, ", activation quantized inside the GEMM" if dynamic else "")
         W = synth.decode_weight(N, K)
         A = synth.decode_activation(M, K)
         self.host = (A, W)
@@ -319,14 +321,19 @@ class DecodeWorkload(Workload):
             D = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
             ws = torch.zeros((max(16, fp4.fp4_gemm_workspace_bytes(fp4.NVFP4, M, N, K)),),
                              dtype=torch.uint8, device=dev)
-            # per call: S_global of the activation, its quantization and alpha in
-            # one launch, then the decode GEMM (the weights were quantized ahead
-            # of time, so it may start streaming them before the quantizer ends)
-            self.calls.append([
-                [fp4.bind_quantize_dynamic(Ad, pA, sA, gA, gW, al, stream)],
-                [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws,
-                               fp4.GEMM_DECODE | fp4.GEMM_B_STATIC, stream)],
-            ])
+            if dynamic:
+                # one call: S_global and alpha (one launch), then the decode GEMM
+                # quantizing each K slice of the activation as it needs it
+                self.calls.append([[fp4.bind_gemm_decode_dynamic(Ad, pW, sW, gW, D, gA, al, ws, stream)]])
+            else:
+                # per call: S_global of the activation, its quantization and alpha in
+                # one launch, then the decode GEMM (the weights were quantized ahead
+                # of time, so it may start streaming them before the quantizer ends)
+                self.calls.append([
+                    [fp4.bind_quantize_dynamic(Ad, pA, sA, gA, gW, al, stream)],
+                    [fp4.bind_gemm(fp4.NVFP4, pA, sA, pW, sW, M, N, K, al, D, ws,
+                                   fp4.GEMM_DECODE | fp4.GEMM_B_STATIC, stream)],
+                ])
             self.bufs.append((pW, sW, Ad, gA, al, pA, sA, D, ws))
         del Wd
         torch.cuda.empty_cache()
@@ -335,8 +342,12 @@ class DecodeWorkload(Workload):
         self.gemm_bytes = wbytes + abytes + M * N * 2
         self.work = {"gemm": self.gemm_bytes, "act_quantize": M * K * 2 + abytes}   # one read of x
         self.bound = {"gemm": "hbm", "act_quantize": "hbm"}
+        if dynamic:
+            # one group: the S_global launch and the GEMM (timed together)
+            self.kernels = ["gemm"]
+            self.work = {"gemm": self.gemm_bytes}
         self.flops = 2.0 * M * N * K
-        self.launches_per_step = 2   # dynamic activation quantizer, decode GEMM
+        self.launches_per_step = 2   # activation quantizer (or S_global), decode GEMM
         self.dominant = "gemm"
         self.l2_note = "rotating %d quantized weight copies (%.0f MB) > %d MB L2" % (
             sets, sets * wbytes / 1e6, L2_BYTES >> 20)
@@ -653,6 +664,8 @@ def make_workload(name, dev, stream):
         return SquareWorkload(fp4.NVFP4, 4096, dev, stream=stream)
     if name.startswith("decode_m"):
         return DecodeWorkload(int(name[len("decode_m"):]), dev, stream=stream)
+    if name.startswith("decode_dyn_m"):
+        return DecodeWorkload(int(name[len("decode_dyn_m"):]), dev, stream=stream, dynamic=True)
     if name == "prefill_up":
         return PrefillWorkload(8192, 28672, 8192, dev, stream=stream)
     if name == "prefill_down":
@@ -673,7 +686,8 @@ def make_workload(name, dev, stream):
     raise SystemExit("unknown workload %r" % name)
 
 
-WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "prefill_up",
+WORKLOADS = ["square_mx", "square_nv", "decode_m1", "decode_m4", "decode_m16", "decode_dyn_m1",
+             "decode_dyn_m4", "decode_dyn_m16", "prefill_up",
              "prefill_down", "moe_grouped_mx", "moe_separate_mx", "dequant_w_nv", "w4a16_prefill_up", "w4a16_decode_m16"] + ["quant_%s_%s_%s" % (s, f, a) for s in ("16384", "8192x28672")
                                 for f in ("nv", "mx", "p1e8") for a in ("row", "col")]
 

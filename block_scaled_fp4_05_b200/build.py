@@ -17,7 +17,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfp4.so")
 SOURCES = ["api.cu", "quantize.cu", "gemm.cu"]
-HEADERS = ["fp4_internal.h"]
+HEADERS = ["fp4_internal.h", "quant_device.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 NVCC_FLAGS = [

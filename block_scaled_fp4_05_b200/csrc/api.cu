@@ -443,6 +443,63 @@ fp4_status fp4_gemm(fp4_format fmt, const void* A, const void* sA, const void* B
                                 FP4_GEMM_AUTO, stream);
 }
 
+fp4_status fp4_gemm_decode_dynamic(const void* act_bf16, int64_t lda, const void* W, const void* sW,
+                                   const float* gsW, int64_t M, int64_t N, int64_t K, void* D,
+                                   int64_t ldd, float* gsA_out, float* alpha_out, void* workspace,
+                                   size_t ws_bytes, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (M < 0 || N < 0 || K < 0 || !gsW || !gsA_out || !alpha_out) return FP4_ERR_INVALID_ARG;
+    if (M > 16) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) {
+        if (ldd < N) return FP4_ERR_INVALID_ARG;
+        return FP4_OK;
+    }
+    if (K == 0 || K % 64 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!act_bf16 || lda < K) return FP4_ERR_INVALID_ARG;
+    if (lda % 8 != 0 || !aligned16(act_bf16) || (reinterpret_cast<uintptr_t>(gsW) & 3u) ||
+        (reinterpret_cast<uintptr_t>(gsA_out) & 3u) || (reinterpret_cast<uintptr_t>(alpha_out) & 3u))
+        return FP4_ERR_MISALIGNED;
+    // the weight side as in fp4_gemm (the packed activation arguments are unused)
+    const fp4_status vs = validate_gemm(FP4_NVFP4, W, sW, W, sW, M, N, K, alpha_out, D, ldd);
+    if (vs != FP4_OK) return vs;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    if (!fp4::tensor_map_encoder_available()) return FP4_ERR_NO_DEVICE;
+    const size_t need = fp4::decode_workspace_bytes(M, N, K, dev.sm_count);
+    if (need == 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (!workspace || ws_bytes < need) return FP4_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return FP4_ERR_MISALIGNED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // S_global of the activation and alpha in one launch, then the GEMM
+    cudaError_t e = fp4::launch_global_scale(static_cast<const uint16_t*>(act_bf16), M, K, lda, gsA_out,
+                                             gsW, alpha_out, s);
+    if (e != cudaSuccess) {
+        fp4::set_last_error("activation S_global launch", e);
+        return from_cuda(e);
+    }
+    fp4::GemmArgs a;
+    a.fmt = fp4::kNv;
+    a.A = nullptr;
+    a.sA = nullptr;
+    a.B = static_cast<const uint8_t*>(W);
+    a.sB = static_cast<const uint8_t*>(sW);
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.alpha = alpha_out;
+    a.D = static_cast<uint16_t*>(D);
+    a.ldd = ldd;
+    a.ws = workspace;
+    a.ws_bytes = ws_bytes;
+    a.b_static = true;
+    a.act = static_cast<const uint16_t*>(act_bf16);
+    a.lda = lda;
+    a.act_gs = gsA_out;
+    return from_cuda(fp4::launch_gemm_decode(a, dev, s));
+}
+
 fp4_status fp4_gemm_decode_noalloc(fp4_format fmt, const void* A, const void* sA, const void* B,
                                    const void* sB, int64_t M, int64_t N, int64_t K,
                                    const float* alpha, void* D, int64_t ldd, fp4_stream_t stream)

@@ -64,6 +64,11 @@ struct GemmArgs {
     void* ws;
     size_t ws_bytes;
     bool b_static;      // B and sB not written by a kernel still running on the stream
+    // decode form only: the activation as BF16 [M x K] (leading dimension
+    // lda), quantized inside the GEMM with S_global *act_gs (A and sA unused)
+    const uint16_t* act = nullptr;
+    int64_t lda = 0;
+    const float* act_gs = nullptr;
 };
 size_t decode_workspace_bytes(int64_t M, int64_t N, int64_t K, int sm_count);
 cudaError_t launch_gemm_prefill(const GemmArgs& a, const DeviceInfo& dev, cudaStream_t s);

@@ -57,6 +57,7 @@
 #include <mutex>
 
 #include "fp4_internal.h"
+#include "quant_device.cuh"
 
 namespace fp4 {
 
@@ -71,7 +72,10 @@ constexpr int MMA_K = 64;           // K per tcgen05.mma for FP4
 constexpr int A_BYTES = BM * BK_BYTES;
 constexpr int SF_CHUNK = 512;       // 128 rows x 4 scale bytes
 constexpr int SFA_BYTES = 4 * SF_CHUNK;
-constexpr int kThreads = 320;    // 10 warps: producer, MMA, 4 epilogue, 4 scale staging
+// 10 warps: producer, MMA, 4 epilogue, 4 scale staging; the decode tile
+// (N = 16) adds 4 activation-quantizer warps
+template <int BN>
+constexpr int kThreadsFor = BN == 16 ? 448 : 320;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 enum : unsigned { ERR_FULL = 1u, ERR_EMPTY = 2u, ERR_ACC_FULL = 4u, ERR_ACC_EMPTY = 8u,
@@ -91,11 +95,17 @@ struct Cfg {
     static constexpr int SFA_COLS = 4 * 4;               // 4 chunks x 4 columns
     static constexpr int SF_COLS = SFA_COLS + 4 * 4 * BH;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    // barriers (1 KB), then, for the decode tile, the activation scale bytes
+    // of each stage formed in the kernel (16 rows x 16 bytes per stage)
+    static constexpr int OFF_ACT = 1024;   // from the barrier area
+    static constexpr int ACT_SF_BYTES = BN == 16 ? STAGES * 256 : 0;
+    static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + OFF_ACT + ACT_SF_BYTES;
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
+    static_assert(SMEM <= 232448, "shared memory per block");
     static_assert(BN % 16 == 0 && BN <= 256, "MMA N");
     static_assert(BH <= 2, "scale staging covers at most two 128-row tiles of B");
-    static_assert((3 * STAGES + 3) * 8 + 8 <= 512, "barrier area");
+    static_assert((3 * STAGES + 3) * 8 + 8 <= 40 * 8, "barrier area below the activation barriers");
+    static_assert((40 + STAGES) * 8 <= OFF_ACT, "activation barriers below the scale buffers");
     static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms stay 1024-aligned");
 };
 
@@ -116,6 +126,12 @@ struct Params {
     int64_t ldd;
     float* ws;
     int* counters;             // stream-K: arrivals per (weight tile, lane quadrant)
+    // decode form with the activation quantized in the kernel (else NULL):
+    // BF16 activation [rows_b x K] with leading dimension lda, and its
+    // S_global (written by the kernel before this one)
+    const uint16_t* act;
+    int64_t lda;
+    const float* act_gs;
 };
 
 // ------------------------------------------------------------------------
@@ -473,7 +489,7 @@ struct Schedule {
 // The kernel
 // ------------------------------------------------------------------------
 template <int BN, int STAGES, int FMT, bool STREAM_K>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreadsFor<BN>, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const Params p)
 {
@@ -494,6 +510,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
     auto full = [&](int s) { return smem_u32(&bars[s]); };
     auto empty = [&](int s) { return smem_u32(&bars[STAGES + s]); };
     auto sf_ready = [&](int s) { return smem_u32(&bars[2 * STAGES + s]); };
+    auto act_full = [&](int s) { return smem_u32(&bars[40 + s]); };
     const uint32_t acc_full = smem_u32(&bars[3 * STAGES]);
     const uint32_t acc_empty = smem_u32(&bars[3 * STAGES + 1]);
     const uint32_t drain = smem_u32(&bars[3 * STAGES + 2]);
@@ -507,6 +524,9 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 4);
         mbar_init(drain, 1);
+        // activation stage published by a quantizer warp (in-kernel
+        // activation quantization, decode tile)
+        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bars[40 + s]), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -542,13 +562,18 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             // K stage ks of segment g into ring slot stg; `expect` posts the
             // stage's full byte count on its barrier.
             auto issue = [&](int stg, const Seg& g, int ks, int nbh, bool a_side, bool b_side, bool expect) {
+                // (b_side is cleared below for an activation quantized in the kernel)
                 const uint32_t fb = bar0 + 8u * stg;
                 const int nk = min(4, (p.K - ks * BK) / MMA_K);
                 const int nch = MX ? nk / 2 : nk;
                 const int ct0 = MX ? ks * 2 : ks * 4;   // first 512-byte scale chunk of the stage
                 const uint32_t sf_bytes = (uint32_t)nch * SF_CHUNK;
                 const uint32_t st = smem0 + stg * C::STAGE_BYTES;
-                if (expect) mbar_arrive_expect_tx(fb, A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
+                const bool dyn = !MX && BN == 16 && p.act != nullptr;   // activation quantized by the staging warps
+                if (expect)
+                    mbar_arrive_expect_tx(fb, dyn ? A_BYTES + sf_bytes
+                                                  : A_BYTES + C::B_BYTES + sf_bytes * (1 + nbh));
+                if (dyn) b_side = false;
                 if (a_side) {
                     tma_load_2d(&tmA, fb, st, ks * BK_BYTES, g.tm * BM);
                     bulk_load(st + C::OFF_SFA, p.sfa + g.tm * sf_row_bytes + ct0 * SF_CHUNK, sf_bytes, fb);
@@ -824,11 +849,16 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             }
             acc_phase ^= 1u;
         }
-    } else {
+    } else if (warp < 10) {
         // ---------------- scale staging (warps 6..9) ----------------
         // Each warp writes its own TMEM lane quadrant: lane l stores the
         // 16-byte row l of every 512-byte chunk (4 consecutive columns).
+        // With an activation quantized in the kernel (decode form, p.act set)
+        // the activation's scale bytes come from the quantizer warps'
+        // per-stage buffer (16 rows x 16 bytes) once act_full[stage] is set.
         const uint32_t tq = tmem_base + ((uint32_t)((warp & 3) * 32) << 16);
+        const bool dyn = !MX && BN == 16 && p.act != nullptr;
+        const uint8_t* act_sf = reinterpret_cast<const uint8_t*>(bars) + C::OFF_ACT;
         Schedule<STREAM_K> sched(p);
         Seg sg;
         int stage = 0;
@@ -841,7 +871,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (rtb0 + h < p.sfb_row_tiles) ++nbh;
             for (int ks = sg.kb; ks < sg.ke; ++ks) {
                 int w = 0;
-                if (lane == 0) w = wait_bounded(full(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
+                if (lane == 0) {
+                    w = wait_bounded(full(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
+                    if (w && dyn) w = wait_fast(act_full(stage), phase, abort_flag, ERR_FULL) ? 1 : 0;
+                }
                 w = __shfl_sync(0xFFFFFFFFu, w, 0);
                 if (!w) {
                     ok = false;
@@ -849,8 +882,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 __syncwarp();
                 tc_fence_after();
-                const int k0 = ks * BK;
-                const int nk = min(4, (p.K - k0) / MMA_K);
+                const int nk = min(4, (p.K - ks * BK) / MMA_K);
                 const int nch = MX ? nk / 2 : nk;
                 const uint32_t st = smem0 + stage * C::STAGE_BYTES + lane * 16;
                 const uint32_t tsf = tq + C::SF_COL0 + stage * C::SF_COLS;
@@ -882,14 +914,29 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     tmem_st32(tsf + C::SFA_COLS, b);
                 } else {
                     uint32_t b[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
+                    if (dyn) {
+                        // lane l < 16 holds activation row l: its word j carries
+                        // blocks 4j..4j+3; the other rows of the chunk are padding
                         uint4 v = make_uint4(0u, 0u, 0u, 0u);
-                        if (j < nch && nbh > 0) v = ld_shared_v4(st + C::OFF_SFB + j * SF_CHUNK);
-                        b[4 * j] = v.x;
-                        b[4 * j + 1] = v.y;
-                        b[4 * j + 2] = v.z;
-                        b[4 * j + 3] = v.w;
+                        if (lane < 16) v = *reinterpret_cast<const uint4*>(act_sf + stage * 256 + lane * 16);
+                        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            b[4 * j] = j < nch ? wv[j] : 0u;
+                            b[4 * j + 1] = 0u;
+                            b[4 * j + 2] = 0u;
+                            b[4 * j + 3] = 0u;
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                            if (j < nch && nbh > 0) v = ld_shared_v4(st + C::OFF_SFB + j * SF_CHUNK);
+                            b[4 * j] = v.x;
+                            b[4 * j + 1] = v.y;
+                            b[4 * j + 2] = v.z;
+                            b[4 * j + 3] = v.w;
+                        }
                     }
                     tmem_st16(tsf + C::SFA_COLS, b);
                 }
@@ -900,6 +947,88 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
+                }
+            }
+        }
+    } else if constexpr (!MX && BN == 16) {
+        // ---------------- activation quantizer (warps 10..13, decode tile) ----------------
+        // With p.act set, warp q = warp - 10 forms the activation operand of
+        // the CTA's stages n = q, q + 4, q + 8, ...: the stage's 16 rows x 256
+        // elements, lane l taking the 32-element chunk c = l % 8 (two
+        // 16-element blocks) of rows l / 8 + 4 j, j = 0..3, quantized exactly
+        // as fp4_quantize does (zero codes and scales outside the matrix).
+        // The 16 code bytes of (row r, chunk c) go to the stage's B slot in
+        // the 128-byte-swizzled layout a TMA load would have produced (16-byte
+        // position c ^ (r % 8) of row r), the two scale bytes to the stage's
+        // scale buffer (row r, bytes 2c, 2c + 1).  The loads and the
+        // arithmetic run before the slot is free; the stores wait for the
+        // MMA of the slot's previous use (the producer's empty barrier), and
+        // the stage is published on act_full[stage].  Four warps take turns,
+        // so the quantization of one stage overlaps that of the next three.
+        if (p.act != nullptr) {
+            pdl_wait();
+            const float gs = *p.act_gs;
+            const float denom = __fmul_rn(6.0f, gs);
+            const int q = warp - 10;
+            const int c = lane & 7;
+            uint8_t* act_sf = reinterpret_cast<uint8_t*>(bars) + C::OFF_ACT;
+            Schedule<STREAM_K> sched(p);
+            Seg sg;
+            int n = 0;
+            bool ok = true;
+            while (ok && sched.next(sg)) {
+                for (int ks = sg.kb; ks < sg.ke; ++ks, ++n) {
+                    if ((n & 3) != q) continue;
+                    const int stage = n % STAGES;
+                    const uint32_t phase = (uint32_t)(n / STAGES) & 1u;
+                    const int k0 = ks * BK;
+                    const int nk = min(4, (p.K - k0) / MMA_K);
+                    uint4 v[4][4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = (lane >> 3) + 4 * j;
+                        const bool in = r < p.rows_b && c < 2 * nk;
+                        const uint4* src =
+                            reinterpret_cast<const uint4*>(p.act + (int64_t)(in ? r : 0) * p.lda + k0 + (in ? c * 32 : 0));
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            v[j][u] = in ? qdev::ld_stream(src + u) : make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    uint4 codes[4];
+                    uint32_t sbw[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float inv0, inv1;
+                        const uint32_t s0 = qdev::block_scale<FMT>(
+                            max(qdev::absmax8(v[j][0]), qdev::absmax8(v[j][1])), gs, denom, &inv0);
+                        const uint32_t s1 = qdev::block_scale<FMT>(
+                            max(qdev::absmax8(v[j][2]), qdev::absmax8(v[j][3])), gs, denom, &inv1);
+                        codes[j] = make_uint4(qdev::quantize8(v[j][0], inv0), qdev::quantize8(v[j][1], inv0),
+                                              qdev::quantize8(v[j][2], inv1), qdev::quantize8(v[j][3], inv1));
+                        sbw[j] = s0 | (s1 << 8);
+                    }
+                    int w = 0;
+                    if (lane == 0) w = wait_bounded(empty(stage), phase ^ 1u, abort_flag, ERR_EMPTY) ? 1 : 0;
+                    w = __shfl_sync(0xFFFFFFFFu, w, 0);
+                    if (!w) {
+                        ok = false;
+                        break;
+                    }
+                    __syncwarp();
+                    const uint32_t slot = smem0 + stage * C::STAGE_BYTES + C::OFF_B;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int r = (lane >> 3) + 4 * j;
+                        const uint32_t dst = slot + r * BK_BYTES + ((uint32_t)(c ^ (r & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(codes[j].x),
+                                     "r"(codes[j].y), "r"(codes[j].z), "r"(codes[j].w)
+                                     : "memory");
+                        *reinterpret_cast<uint16_t*>(act_sf + stage * 256 + r * 16 + c * 2) = (uint16_t)sbw[j];
+                    }
+                    // the codes are read by the tensor core (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(act_full(stage));
                 }
             }
         }
@@ -1597,7 +1726,7 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Pa
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.blockDim = dim3(kThreadsFor<BN>, 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -1702,6 +1831,9 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.ldd = a.ldd;
     p.ws = nullptr;
     p.counters = nullptr;
+    p.act = nullptr;
+    p.lda = 0;
+    p.act_gs = nullptr;
     p.units = 0;
     p.sk_tiles = 0;
     p.a_static = 0;
@@ -1818,7 +1950,10 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     // swap: the weight operand B [N x K] is the 128-row MMA side, the M <= 16
     // tokens form the N = 16 side
     CUtensorMap tw, tx;
-    if (!make_map(&tw, a.B, a.N, a.K / 2, BM) || !make_map(&tx, a.A, a.M, a.K / 2, DECODE_BN)) {
+    // (with the activation quantized in the kernel there is no packed
+    // activation to map: the weights' map is passed in its place, unused)
+    if (!make_map(&tw, a.B, a.N, a.K / 2, BM) ||
+        !make_map(&tx, a.act ? a.B : a.A, a.act ? a.N : a.M, a.K / 2, DECODE_BN)) {
         set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return cudaErrorInvalidValue;
     }
@@ -1830,6 +1965,9 @@ cudaError_t launch_gemm_decode(const GemmArgs& a, const DeviceInfo& dev, cudaStr
     const int G = d.G;
     p.sk_tiles = d.sk_tiles;
     p.a_static = a.b_static ? 1 : 0;   // the weight operand B is the MMA A side here
+    p.act = a.act;
+    p.lda = a.lda;
+    p.act_gs = a.act_gs;
     p.units = d.sk_tiles * p.ks_total;
     p.max_seg = d.max_seg;
     // the counters start at zero (caller's contract) and the kernel leaves

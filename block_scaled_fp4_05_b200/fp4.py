@@ -85,6 +85,8 @@ def lib():
         L.fp4_get_device_status.argtypes = [st]
         L.fp4_selftest_bounded_wait.restype = c.c_int
         L.fp4_selftest_bounded_wait.argtypes = [st]
+        L.fp4_gemm_decode_dynamic.restype = c.c_int
+        L.fp4_gemm_decode_dynamic.argtypes = [P, i64, P, P, P, i64, i64, i64, P, i64, P, P, P, sz, st]
         L.fp4_gemm_decode_noalloc.restype = c.c_int
         L.fp4_gemm_decode_noalloc.argtypes = [c.c_int, P, P, P, P, i64, i64, i64, P, P, i64, st]
         _lib = L
@@ -282,6 +284,28 @@ def fp4_gemm(fmt, A, sA, B, sB, M, N, K, alpha, D, workspace=None, kernel=GEMM_A
                                       _dptr(workspace, "workspace"), ws_bytes, int(kernel),
                                       _stream(stream)),
            "fp4_gemm")
+
+
+def fp4_gemm_decode_dynamic(x, W, sW, gsW, D, gs_out, alpha_out, workspace, stream=None):
+    """NVFP4 decode GEMM quantizing the BF16 activation x [M x K] inside the
+    kernel: gs_out = S_global(x), alpha_out = gs_out * gsW, D = alpha * x_hat W_hat^T."""
+    assert x.dtype == torch.bfloat16
+    M, K = x.shape
+    N = W.shape[0]
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().fp4_gemm_decode_dynamic(_dptr(x, "x"), _ld(x), _dptr(W, "W"), _dptr(sW, "sW"),
+                                         _dptr(gsW, "gsW"), M, N, K, _dptr(D, "D"), D.stride(0),
+                                         _dptr(gs_out, "gs_out"), _dptr(alpha_out, "alpha_out"),
+                                         _dptr(workspace, "workspace"), ws_bytes, _stream(stream)),
+           "fp4_gemm_decode_dynamic")
+
+
+def bind_gemm_decode_dynamic(x, W, sW, gsW, D, gs_out, alpha_out, workspace, stream=None):
+    M, K = x.shape
+    return BoundCall("fp4_gemm_decode_dynamic", _dptr(x, "x"), _ld(x), _dptr(W, "W"), _dptr(sW, "sW"),
+                     _dptr(gsW, "gsW"), M, W.shape[0], K, _dptr(D, "D"), D.stride(0),
+                     _dptr(gs_out, "gs_out"), _dptr(alpha_out, "alpha_out"), _dptr(workspace, "workspace"),
+                     workspace.numel() * workspace.element_size(), _stream(stream))
 
 
 def fp4_get_device_status(stream=None):

@@ -325,6 +325,40 @@ fp4_status fp4_gemm_grouped(fp4_format fmt, int n, const fp4_gemm_problem* probl
 size_t fp4_gemm_workspace_bytes(fp4_format fmt, int64_t M, int64_t N, int64_t K);
 
 /*
+ * Decode GEMM with the activation quantized inside the GEMM (NVFP4):
+ *   S_global,A = amax|A| / 2688 (1 if zero)      -> *gsA_out
+ *   alpha      = S_global,A * (*gsW)             -> *alpha_out
+ *   D          = alpha * A_hat * W_hat^T (BF16)
+ * where A_hat is the NVFP4 quantization of the BF16 activation A with
+ * S_global,A (identical bytes to fp4_quantize_dynamic), formed block by
+ * block in shared memory by the GEMM kernel itself as its K slices are
+ * needed, never written to global memory.  Two launches: the one-launch
+ * S_global/alpha kernel, then the decode GEMM, which streams its first
+ * weight tiles while the first launch runs.  Every thread block quantizes
+ * the activation slices its own K range needs, so for this path the BF16
+ * activation (4x the bytes of its packed form) is read from L2 by every
+ * block; fp4_quantize_dynamic followed by fp4_gemm is the faster decode
+ * when the activation can go through global memory.  [NVFP4-Arch] "1. The
+ * Dual-Level Mathematical Formulation" (per-tensor and block scales of an
+ * activation quantized on the fly) and "2. Hardware-Managed Tensor Core
+ * Dot-Products".
+ *   act_bf16 : device, BF16 [M x K], leading dimension lda (elements)
+ *   W, sW    : device, the packed NVFP4 weights [N x K/2] and their scales,
+ *              quantized ahead of time with S_global *gsW; W, sW and gsW
+ *              must not be written by a kernel still running on the stream
+ *   D        : BF16 [M x N], leading dimension ldd
+ *   gsA_out, alpha_out : device floats, written
+ *   workspace / ws_bytes : as for fp4_gemm's decode kernel
+ *              (fp4_gemm_workspace_bytes(FP4_NVFP4, M, N, K)), counters zero
+ * Requires 1 <= M <= 16 (else FP4_ERR_UNSUPPORTED_SHAPE), K % 64 == 0,
+ * N % 8 == 0, lda % 8 == 0; M == 0 or N == 0 is a no-op.
+ */
+fp4_status fp4_gemm_decode_dynamic(const void* act_bf16, int64_t lda, const void* W, const void* sW,
+                                   const float* gsW, int64_t M, int64_t N, int64_t K, void* D,
+                                   int64_t ldd, float* gsA_out, float* alpha_out, void* workspace,
+                                   size_t ws_bytes, fp4_stream_t stream);
+
+/*
  * Allocation-free form of the decode GEMM (no counterpart on the pages: it is
  * a service of this library, not part of the method).  Same operation,
  * arguments, result and kernels as fp4_gemm_with_kernel(..., FP4_GEMM_DECODE),

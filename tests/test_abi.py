@@ -173,3 +173,20 @@ def test_global_scale_alpha_host_checks_without_gpu():
     assert f(A16, 4, 8, 8, A16, A16, P((1 << 20) + 2), None) == 3   # misaligned alpha
     if not torch.cuda.is_available():
         assert f(A16, 4, 8, 8, A16, A16, A16, None) == 6
+
+
+def test_decode_dynamic_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    f = L.fp4_gemm_decode_dynamic
+    ws = P(1 << 24)
+    # (act, lda, W, sW, gsW, M, N, K, D, ldd, gs_out, alpha_out, ws, ws_bytes, stream)
+    assert f(A16, 64, A16, A16, None, 4, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 1   # no gsW
+    assert f(A16, 64, A16, A16, A16, 17, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 2   # M > 16
+    assert f(A16, 96, A16, A16, A16, 4, 16, 96, A16, 16, A16, A16, ws, 1 << 20, None) == 2    # K % 64
+    assert f(None, 64, A16, A16, A16, 4, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 1   # no activation
+    assert f(A16, 32, A16, A16, A16, 4, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 1    # lda < K
+    assert f(A1, 64, A16, A16, A16, 4, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 3     # misaligned
+    assert f(A16, 64, A16, A16, A16, 0, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 0    # M == 0: no-op
+    if not torch.cuda.is_available():
+        assert f(A16, 64, A16, A16, A16, 4, 16, 64, A16, 16, A16, A16, ws, 1 << 20, None) == 6
