@@ -150,91 +150,99 @@ quantize_rowwise_tiles_kernel(const __grid_constant__ RowBatch b)
 // even: the product of the E2M1 value, the block scale and S_global is exact
 // in FP64 (at most 2 + 4 + 24 significant bits), then converted.  HBM-bound
 // (0.5 + 1/blk bytes read, 2 written per element).
-// A warp takes 1024 consecutive codes of one row (4 segments of 256): in each
+// Each block first tabulates, for all 256 scale bytes, the BF16 results of
+// the eight E2M1 magnitudes times that scale (exact FP64 product, one
+// rounding): the low bytes of magnitudes 0..7 in 8 bytes, the high bytes in
+// 8 more.  A code's magnitude (3 bits) is then directly a byte-permute
+// selector: one permute yields the high (or low) bytes of four codes, the
+// code signs flip bit 7 of the high bytes, and two more permutes interleave
+// low and high bytes into BF16 pairs.
+// A warp takes 2048 consecutive codes of one row (8 segments of 256): in each
 // segment lane l owns codes [8l, 8l + 8), one 4-byte load of packed codes and
 // one 16-byte store of BF16, so every warp load covers 128 contiguous bytes
-// and every warp store 512.  The 8 magnitudes of a block's scale (the
-// rounding table) are computed by two neighbouring lanes, four each, and
-// exchanged with shuffles.
+// and every warp store 512.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t bf16_bits_rn(double x)
+{
+    unsigned short h;
+    asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(h) : "d"(x));
+    return h;
+}
+
+// Eight E2M1 codes (code i in bits 4i..4i+3 of w) to BF16 through the table
+// entry tb of their block's scale byte (x, y: low bytes of magnitudes 0..3,
+// 4..7; z, w: high bytes): output word i holds codes 2i (low half) and 2i + 1.
+__device__ __forceinline__ uint4 decode8(uint32_t w, uint4 tb)
+{
+    const uint32_t sel0 = w & 0x7777u;            // magnitudes of codes 0..3
+    const uint32_t sel1 = (w >> 16) & 0x7777u;    // codes 4..7
+    const uint32_t l0 = __byte_perm(tb.x, tb.y, sel0), l1 = __byte_perm(tb.x, tb.y, sel1);
+    uint32_t h0 = __byte_perm(tb.z, tb.w, sel0), h1 = __byte_perm(tb.z, tb.w, sel1);
+    // sign of code 2j (2j + 1) in bit 7 of byte j of ev (od)
+    const uint32_t ev = (w << 4) & 0x80808080u, od = w & 0x80808080u;
+    h0 ^= __byte_perm(ev, od, 0x5140);
+    h1 ^= __byte_perm(ev, od, 0x7362);
+    return make_uint4(__byte_perm(l0, h0, 0x5140), __byte_perm(l0, h0, 0x7362), __byte_perm(l1, h1, 0x5140),
+                      __byte_perm(l1, h1, 0x7362));
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(kThreads)
 dequantize_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ scales,
                   const float* __restrict__ gs_ptr, int64_t rows, int64_t k, uint16_t* __restrict__ out,
                   int64_t ld)
 {
+    static_assert(kThreads == 256, "one table entry per thread");
     pdl_trigger();
     constexpr int KB = FMT == kMx ? 32 : 16;
+    constexpr int CPT = 4 * KB;                         // codes per 512-byte scale tile column
     constexpr int SEG = 256;                            // codes per warp segment
-    constexpr int UNROLL = 4;
-    const double gs = FMT != kMx ? (double)__ldg(gs_ptr) : 1.0;
+    constexpr int UNROLL = 8;
+    __shared__ uint4 s_tab[256];
+    {
+        const uint32_t byte = threadIdx.x;
+        const double gs = FMT != kMx ? (double)__ldg(gs_ptr) : 1.0;
+        const double s = FMT == kNv ? (double)e4m3_value(byte)
+                                    : __longlong_as_double((long long)(byte + 896) << 52);  // 2^(byte - 127)
+        const double eff = s * gs;
+        const double q[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+        uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint32_t b = bf16_bits_rn(q[m] * eff);
+            lo[m / 4] |= (b & 0xFFu) << (8 * (m % 4));
+            hi[m / 4] |= (b >> 8) << (8 * (m % 4));
+        }
+        s_tab[byte] = make_uint4(lo[0], lo[1], hi[0], hi[1]);
+    }
+    __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int64_t nsc = k / KB;                         // scales per row
-    const int64_t nct = (nsc + 3) / 4;                  // scale tiles per 128-row group
+    const int64_t nct = (k / KB + 3) / 4;               // scale tile columns per 128-row group
     const int64_t groups_per_row = (k + SEG * UNROLL - 1) / (SEG * UNROLL);
     const int64_t total = rows * groups_per_row;
     const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
-    const int half = lane & 1;                          // which four table entries this lane forms
+    // this lane's scale byte within a segment: tile column, then block in it
+    const int lane_sc = ((lane * 8) / CPT) * 512 + ((lane * 8) / KB) % 4;
     for (int64_t w = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); w < total; w += warps) {
         const int64_t r = w / groups_per_row;
-        const int64_t c_base = (w - r * groups_per_row) * (SEG * UNROLL);
-        const uint8_t* prow = packed + r * (k / 2);
-        const uint8_t* srow = scales + (r / 128) * nct * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4;
+        const int c_base = (int)(w - r * groups_per_row) * (SEG * UNROLL);
+        const uint32_t* prow = reinterpret_cast<const uint32_t*>(packed + r * (k / 2) + c_base / 2) + lane;
+        const uint8_t* srow = scales + (r / 128) * nct * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 +
+                              (int64_t)(c_base / CPT) * 512 + lane_sc;
+        uint16_t* orow = out + r * ld + c_base + lane * 8;
+        const int64_t rem = k - c_base;                 // codes of the row from c_base on
+        const int left = (int)(rem < SEG * UNROLL ? rem : SEG * UNROLL) - lane * 8;
         uint32_t words[UNROLL];
-        uint8_t sbytes[UNROLL];
+        uint32_t sbytes[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            const int64_t c0 = c_base + u * SEG + lane * 8;    // first code of this lane
-            const bool in = c0 < k;
-            words[u] = in ? __ldg(reinterpret_cast<const uint32_t*>(prow + c0 / 2)) : 0u;
-            const int64_t blk = c0 / KB;
-            sbytes[u] = in ? __ldg(srow + (blk / 4) * 512 + blk % 4) : (uint8_t)0;
+            const bool in = u * SEG < left;
+            words[u] = in ? __ldg(prow + u * (SEG / 8)) : 0u;
+            sbytes[u] = in ? __ldg(srow + u * (SEG / CPT) * 512) : 0u;
         }
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-            const int64_t c0 = c_base + u * SEG + lane * 8;
-            double s;
-            if (FMT == kNv) {
-                s = (double)e4m3_value(sbytes[u]);
-            } else {
-                s = __longlong_as_double((long long)(sbytes[u] + 896) << 52);   // 2^(byte - 127), exact
-            }
-            const double eff = s * gs;
-            // this lane's four entries of the table, the neighbour's four by shuffle
-            // E2M1 magnitudes 0, .5, 1, 1.5 (even lane) or 2, 3, 4, 6 (odd lane)
-            const double q0 = half ? 2.0 : 0.0, q1 = half ? 3.0 : 0.5;
-            const double q2 = half ? 4.0 : 1.0, q3 = half ? 6.0 : 1.5;
-            uint32_t mine[2], other[2];
-            mine[0] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(q0 * eff)) |
-                      ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(q1 * eff)) << 16);
-            mine[1] = (uint32_t)__bfloat16_as_ushort(__double2bfloat16(q2 * eff)) |
-                      ((uint32_t)__bfloat16_as_ushort(__double2bfloat16(q3 * eff)) << 16);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) other[j] = __shfl_xor_sync(0xFFFFFFFFu, mine[j], 1);
-            // magnitudes 0..7 as BF16 pairs: t[0] = {0, 1}, t[1] = {2, 3}, ...
-            // (both lanes of a pair hold the same block: 8 codes per lane and
-            // at least 16 per block)
-            const uint32_t t0 = half ? other[0] : mine[0];
-            const uint32_t t1 = half ? other[1] : mine[1];
-            const uint32_t t2 = half ? mine[0] : other[0];
-            const uint32_t t3 = half ? mine[1] : other[1];
-            auto lookup = [&](uint32_t nib) {
-                const uint32_t lo = (nib & 2u) ? t1 : t0;
-                const uint32_t hi = (nib & 2u) ? t3 : t2;
-                const uint32_t w2 = (nib & 4u) ? hi : lo;
-                const uint32_t mag = (nib & 1u) ? (w2 >> 16) : (w2 & 0xFFFFu);
-                return mag | ((nib & 8u) << 12);
-            };
-            if (c0 < k) {
-                uint32_t o[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t byte = (words[u] >> (8 * i)) & 0xFFu;
-                    o[i] = lookup(byte & 0xFu) | (lookup(byte >> 4) << 16);
-                }
-                *reinterpret_cast<uint4*>(out + r * ld + c0) = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-        }
+        for (int u = 0; u < UNROLL; ++u)
+            if (u * SEG < left) *reinterpret_cast<uint4*>(orow + u * SEG) = decode8(words[u], s_tab[sbytes[u]]);
     }
 }
 
@@ -717,6 +725,32 @@ cudaError_t launch_quantize_rowwise_batch(int fmt, int n, const RowwiseDesc* d, 
     return cudaSuccess;
 }
 
+// Resident blocks per SM of the dequantizer (per device and format, looked
+// up once).
+int dequantize_blocks_per_sm(int fmt)
+{
+    static std::mutex mu;
+    static int cache[64][3] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 4;
+    }
+    const int f = fmt == kNv ? 0 : fmt == kP1 ? 1 : 2;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev][f]) return cache[dev][f];
+    int nb = 0;
+    cudaError_t e = fmt == kNv ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, dequantize_kernel<kNv>, kThreads, 0)
+                  : fmt == kP1 ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, dequantize_kernel<kP1>, kThreads, 0)
+                               : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, dequantize_kernel<kMx>, kThreads, 0);
+    if (e != cudaSuccess || nb < 1) {
+        cudaGetLastError();
+        nb = 4;
+    }
+    if (dev < 64) cache[dev][f] = nb;
+    return nb;
+}
+
 cudaError_t launch_dequantize(int fmt, const uint8_t* packed, const uint8_t* scales, const float* gs,
                               int64_t rows, int64_t k, uint16_t* out, int64_t ld, cudaStream_t s)
 {
@@ -724,9 +758,12 @@ cudaError_t launch_dequantize(int fmt, const uint8_t* packed, const uint8_t* sca
     DeviceInfo dev;
     cudaError_t e = device_info(&dev);
     if (e != cudaSuccess) return e;
-    const int64_t warps = rows * ((k + 1023) / 1024);
+    // one warp per 2048 codes of a row, at most one wave of resident blocks
+    // (every block gets the same share of a grid-stride loop, so a second,
+    // partial wave would double the time of the blocks in it)
+    const int64_t warps = rows * ((k + 2047) / 2048);
     int64_t grid = (warps + kThreads / 32 - 1) / (kThreads / 32);
-    const int64_t cap = (int64_t)dev.sm_count * 8;
+    const int64_t cap = (int64_t)dev.sm_count * dequantize_blocks_per_sm(fmt);
     if (grid > cap) grid = cap;
     if (fmt == kNv)
         dequantize_kernel<kNv><<<(unsigned)grid, kThreads, 0, s>>>(packed, scales, gs, rows, k, out, ld);

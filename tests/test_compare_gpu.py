@@ -25,7 +25,8 @@ def f64_to_bf16_bits(x):
     _, e = np.frexp(a)
     q_exp = np.where(e - 1 >= -126, e - 8, -133)      # quantum: 8 significant bits, or subnormal
     v = np.ldexp(np.round(np.ldexp(a, -q_exp)), q_exp)
-    bits = (v.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    with np.errstate(over="ignore"):              # beyond the BF16 range: infinity
+        bits = (v.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
     return np.where(neg, bits | 0x8000, bits).astype(np.uint16)
 
 
@@ -48,6 +49,32 @@ def test_dequantize_matches_oracle(orc, fmt, shape):
     want = f64_to_bf16_bits(orc.dequantize(fmt, p, s, gs=gs).reshape(rows, K))
     out = torch.full((rows, K + 8), float("nan"), dtype=torch.bfloat16, device="cuda")
     fp4.fp4_dequantize(fmt, to_dev_u8(p), to_dev_u8(s), to_dev_f32(gs) if fmt != fp4.MXFP4 else None,
+                       out[:, :K])
+    torch.cuda.synchronize()
+    got = out[:, :K].cpu().view(torch.int16).numpy().view(np.uint16)
+    bad = np.argwhere(got != want)
+    assert bad.size == 0, (bad[:4].tolist(), got[tuple(bad[0])], want[tuple(bad[0])])
+    assert torch.isnan(out[:, K:].float()).all()
+
+
+@pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4, fp4.P1E8])
+@pytest.mark.parametrize("gs", [0.37, 3.1e-38, 2.0e36])
+def test_dequantize_random_codes_and_scales(orc, fmt, gs):
+    # every code with scale bytes drawn over the whole encoding (negative and
+    # subnormal E4M3, E8M0 0..255; not the E4M3 NaN codes) and S_global
+    # values whose products underflow to BF16 subnormals or overflow: the
+    # rounding of every product, not only of the quantizer's usual range
+    rows, K = 130, 1024
+    rng = np.random.default_rng(63 + fmt)
+    p = rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+    nb = fp4.fp4_scale_bytes(fmt, rows, K)
+    s = rng.integers(0, 256, size=nb, dtype=np.uint8)
+    if fmt == fp4.NVFP4:
+        s[(s & 0x7F) == 0x7F] = 0x3F
+    g = gs if fmt != fp4.MXFP4 else 0.0
+    want = f64_to_bf16_bits(orc.dequantize(fmt, p, s, gs=g).reshape(rows, K))
+    out = torch.full((rows, K + 8), float("nan"), dtype=torch.bfloat16, device="cuda")
+    fp4.fp4_dequantize(fmt, to_dev_u8(p), to_dev_u8(s), to_dev_f32(g) if fmt != fp4.MXFP4 else None,
                        out[:, :K])
     torch.cuda.synchronize()
     got = out[:, :K].cpu().view(torch.int16).numpy().view(np.uint16)
