@@ -1204,11 +1204,12 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uin
     }
 }
 
-// Instruction descriptor of the pair MMA: M = 256 (128 rows per CTA), N = 256.
+// Instruction descriptor of the pair MMA: M = 256 (128 rows per CTA), N = 256
+// (or 128 for a half tile).
 template <int FMT>
-__device__ __forceinline__ uint32_t make_idesc_pair(uint32_t sf_id)
+__device__ __forceinline__ uint32_t make_idesc_pair(uint32_t sf_id, uint32_t n = PAIR_BN)
 {
-    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(PAIR_BN >> 3) << 17) |
+    return (sf_id << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) |
            ((FMT != kNv ? 1u : 0u) << 23) | ((uint32_t)(256 >> 4) << 24) | (sf_id << 29);
 }
 
@@ -1264,6 +1265,9 @@ struct PairArgs {
     Params p[NG];
     int n;
     int tile_begin[NG + 1];
+    // launch tiles from split_from on (a last, partial wave) are computed as
+    // two 256 x 128 halves each, on two pairs (== tile_begin[n]: no split)
+    int split_from;
 };
 
 template <int STAGES, int FMT, int NG>
@@ -1321,13 +1325,23 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
 
     const int pair = blockIdx.x >> 1;
     const int npairs = gridDim.x >> 1;
-    const int tiles = args.tile_begin[args.n];
-    // problem and its local tile index of launch tile t
-    auto locate = [&](int t, int& g, int& lt) {
+    // work items: whole tiles below split_from, then two halves per tile
+    const int tiles = args.split_from + 2 * (args.tile_begin[args.n] - args.split_from);
+    // problem, M and N tile of work item t, and its column half: nh = 0 for a
+    // whole 256 x 256 tile, 1 + h for the columns [128 h, 128 h + 128) of it
+    auto locate = [&](int t, int& g, int& tm, int& tn, int& nh) {
+        int ft = t;
+        nh = 0;
+        if (t >= args.split_from) {
+            ft = args.split_from + ((t - args.split_from) >> 1);
+            nh = 1 + ((t - args.split_from) & 1);
+        }
         g = 0;
         if (NG > 1)
-            while (g + 1 < args.n && t >= args.tile_begin[g + 1]) ++g;
-        lt = t - args.tile_begin[g];
+            while (g + 1 < args.n && ft >= args.tile_begin[g + 1]) ++g;
+        const int lt = ft - args.tile_begin[g];
+        tm = lt % args.p[g].tiles_m;
+        tn = lt / args.p[g].tiles_m;
     };
 
     if (warp == 0) {
@@ -1342,20 +1356,22 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             bool ok = true;
             pdl_wait();
             for (int t = pair; ok && t < tiles; t += npairs) {
-                int g, lt;
-                locate(t, g, lt);
+                int g, tm, tn, nh;
+                locate(t, g, tm, tn, nh);
                 const Params& p = args.p[g];
                 const int64_t sf_row_bytes = (int64_t)p.sf_col_tiles * SF_CHUNK;
-                const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
                 const int rta = tm * 2 + (int)rank;                // this CTA's 128-row A tile
                 const bool has_sfa = rta < p.sfa_row_tiles;
+                // B rows of the item: a half tile has the 128 from column
+                // 128 h, each CTA's 64 the first rows of its 128-row box
+                const int rtb0 = nh ? tn * 2 + nh - 1 : tn * 2;
                 int nbh = 0;
-                for (int h = 0; h < 2; ++h)
-                    if (tn * 2 + h < p.sfb_row_tiles) ++nbh;
+                for (int h = 0; h < (nh ? 1 : 2); ++h)
+                    if (rtb0 + h < p.sfb_row_tiles) ++nbh;
                 const uint8_t* sfa_row = p.sfa + rta * sf_row_bytes;
-                const uint8_t* sfb_row = p.sfb + (int64_t)(tn * 2) * sf_row_bytes;
+                const uint8_t* sfb_row = p.sfb + (int64_t)rtb0 * sf_row_bytes;
                 const int ya = rta * BM;
-                const int yb = tn * PAIR_BN + (int)rank * PAIR_BHALF;
+                const int yb = nh ? rtb0 * 128 + (int)rank * (PAIR_BHALF / 2) : tn * PAIR_BN + (int)rank * PAIR_BHALF;
                 for (int ks = 0; ks < p.ks_total; ++ks) {
                     if (!wait_fast(B_EMPTY(stage), phase ^ 1u, abort_flag, ERR_EMPTY)) {
                         ok = false;
@@ -1406,18 +1422,19 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             const uint64_t adesc0 = desc_sw128(smem0);
             const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
             constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;
-            const uint32_t idesc0 = make_idesc_pair<FMT>(0);
-            const uint32_t idesc2 = make_idesc_pair<FMT>(2);
             const uint32_t tsf0 = tmem_base + C::SF_COL0;
             int stage = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             int pending = -1;   // stage whose release commit is still to be issued
             for (int t = pair; ok && t < tiles; t += npairs) {
-                int g, lt;
-                locate(t, g, lt);
+                int g, tm, tn, nh;
+                locate(t, g, tm, tn, nh);
                 const Params& p = args.p[g];
                 const int kst = p.ks_total;
+                const uint32_t n_mma = nh ? PAIR_BN / 2 : PAIR_BN;
+                const uint32_t idesc0 = make_idesc_pair<FMT>(0, n_mma);
+                const uint32_t idesc2 = make_idesc_pair<FMT>(2, n_mma);
                 if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY) ||
                     !wait_fast(B_FULL(stage), phase, abort_flag, ERR_FULL)) {
                     ok = false;
@@ -1483,12 +1500,26 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
         const uint32_t acc_empty_leader = map_to_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
         for (int t = pair; t < tiles; t += npairs) {
-            int g, lt;
-            locate(t, g, lt);
+            int g, tm, tn, nh;
+            locate(t, g, tm, tn, nh);
             const Params& p = args.p[g];
             const float alpha = p.alpha ? *p.alpha : 1.0f;
             if (!warp_wait(acc_full, acc_phase, abort_flag, ERR_ACC_FULL)) break;
             tc_fence_after();
+            if (nh && half) {
+                // a half tile has 128 accumulator columns: the second-half
+                // warps only hand the accumulator back
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (leader)
+                        mbar_arrive(acc_empty);
+                    else
+                        mbar_arrive_cluster_relaxed(acc_empty_leader);
+                }
+                acc_phase ^= 1u;
+                continue;
+            }
             // four 32-column loads, two buffers: each load overlaps the
             // conversion of the previous chunk
             uint32_t packed[64];
@@ -1523,15 +1554,15 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             // time go to its staging block (64-byte rows; 16-byte chunk j of
             // row r at chunk j ^ ((r >> 1) & 3), the 64-byte swizzle), then
             // one lane stores the block with TMA, coalesced and clipped to D.
-            const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
             const int y0 = (tm * 2 + (int)rank) * BM + q * 32;
+            const int col0 = nh ? tn * PAIR_BN + (nh - 1) * 128 : tn * PAIR_BN + half * 128;
             const uint32_t blk = smem0 + C::OFF_EPI + eb * C::EPI_BLOCK;
             const uint32_t my_row = blk + lane * 64;
             const int sw = (lane >> 1) & 3;
             if (y0 < p.rows_a) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int x0 = tn * PAIR_BN + half * 128 + c * 32;
+                    const int x0 = col0 + c * 32;
                     if (x0 >= p.rows_b) break;
                     if (lane == 0) bulk_wait_read_all();   // the block's previous store has read it
                     __syncwarp();
@@ -1558,14 +1589,15 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
         uint32_t phase = 0;
         bool ok = true;
         for (int t = pair; ok && t < tiles; t += npairs) {
-            int g, lt;
-            locate(t, g, lt);
+            int g, tm, tn, nh;
+            locate(t, g, tm, tn, nh);
             const Params& p = args.p[g];
-            const int tm = lt % p.tiles_m, tn = lt / p.tiles_m;
             const bool has_sfa = tm * 2 + (int)rank < p.sfa_row_tiles;
+            // scale row tiles of B staged (a half tile has one)
+            const int rtb0 = nh ? tn * 2 + nh - 1 : tn * 2;
             int nbh = 0;
-            for (int h = 0; h < 2; ++h)
-                if (tn * 2 + h < p.sfb_row_tiles) ++nbh;
+            for (int h = 0; h < (nh ? 1 : 2); ++h)
+                if (rtb0 + h < p.sfb_row_tiles) ++nbh;
             for (int ks = 0; ks < p.ks_total; ++ks) {
                 if (!warp_wait(B_SFFULL(stage), phase, abort_flag, ERR_FULL)) {
                     ok = false;
@@ -1899,12 +1931,21 @@ bool fill_pair_problem(PairArgs<NG>& args, int g, const GemmArgs& a)
 }
 
 template <int NG>
-cudaError_t launch_pair(const PairArgs<NG>& args, int fmt, const DeviceInfo& dev, cudaStream_t s)
+cudaError_t launch_pair(PairArgs<NG>& args, int fmt, const DeviceInfo& dev, cudaStream_t s)
 {
     const int64_t tiles = args.tile_begin[args.n];
     if (tiles == 0) return cudaSuccess;
     const int64_t max_pairs = dev.sm_count / 2;
-    const int grid = 2 * (int)(tiles < max_pairs ? tiles : max_pairs);
+    // Tiles are dealt to the pairs round-robin, so a last wave of R < pairs
+    // tiles leaves pairs idle for a whole tile.  When its halves fit on the
+    // pairs (2R <= pairs) those R tiles are computed as 2R half tiles
+    // (256 x 128), one per pair.  (A stage's fixed latency makes a half tile
+    // take more than half a tile's time; the split still shortens the wave.)
+    const int64_t rem = tiles % max_pairs;
+    const bool split = NG == 1 && rem > 0 && 2 * rem <= max_pairs;
+    args.split_from = (int)(split ? tiles - rem : tiles);
+    const int64_t items = tiles + (split ? rem : 0);
+    const int grid = 2 * (int)(items < max_pairs ? items : max_pairs);
     if (fmt == kMx) return launch_pair_kernel<PAIR_STAGES_MX, kMx, NG>(args, grid, s);
     if (fmt == kP1) return launch_pair_kernel<PAIR_STAGES_NV, kP1, NG>(args, grid, s);
     return launch_pair_kernel<PAIR_STAGES_NV, kNv, NG>(args, grid, s);

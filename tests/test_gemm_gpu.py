@@ -246,8 +246,22 @@ def sampled_check(orc, fmt, A_bits, B_bits, kernel, n_pairs=4096):
 
 @pytest.mark.parametrize("fmt", FMTS)
 def test_square_4096_sampled(orc, fmt):
+    # 256 tiles over 74 CTA pairs: the 34 tiles of the last wave run as 68
+    # half tiles (256 x 128)
     A, B = synth.square(4096)
     sampled_check(orc, fmt, A, B, fp4.GEMM_PREFILL)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_prefill_tail_halves_ragged(orc, fmt):
+    # 8 x 11 = 88 tiles with both edges ragged (M = 2000, N = 2600): the 14
+    # tiles of the last wave are split into column halves, the last of them
+    # only 40 columns wide; the samples cover every output row and column
+    # range, the split tiles included
+    M, N, K = 2000, 2600, 1024
+    A = synth.normal_bf16(M, K, seed=71, outlier_factor=100.0)
+    B = synth.normal_bf16(N, K, seed=71, tensor_id=1, sigma=0.02)
+    sampled_check(orc, fmt, A, B, fp4.GEMM_PREFILL, n_pairs=8192)
 
 
 @pytest.mark.parametrize("M", [1, 4, 16])
