@@ -203,8 +203,7 @@ class SquareWorkload(Workload):
                 gA = torch.empty(1, dtype=torch.float32, device=dev)
                 gB = torch.empty(1, dtype=torch.float32, device=dev)
                 al = torch.empty(1, dtype=torch.float32, device=dev)
-                groups.append([fp4.bind_global_scale(Ad, gA, stream),
-                               fp4.bind_global_scale_alpha(Bd, gB, gA, al, stream)])
+                groups.append([fp4.bind_global_scales_pair(Ad, Bd, gA, gB, al, stream)])
             else:
                 gA = gB = al = None
             groups.append([fp4.bind_quantize_batch(fmt, [(Ad, pA, sA, gA), (Bd, pB, sB, gB)], stream)])
@@ -216,7 +215,7 @@ class SquareWorkload(Workload):
         self.work = {"quantize": 2 * qbytes, "gemm": 2.0 * n ** 3, "global_scales": 2.0 * n * n * 2}
         self.bound = {"quantize": "hbm", "gemm": "tensor", "global_scales": "hbm"}
         self.flops = 2.0 * n ** 3
-        self.launches_per_step = 2 if fmt == fp4.MXFP4 else 4
+        self.launches_per_step = 2 if fmt == fp4.MXFP4 else 3
         self.dominant = "gemm"
         self.l2_note = "rotating %d input sets (%.0f MB of BF16 inputs) > %d MB L2" % (
             sets, sets * 4 * n * n / 1e6, L2_BYTES >> 20)
@@ -236,10 +235,10 @@ class SquareWorkload(Workload):
         Ad = self.hA.to(dev, non_blocking=True)
         Bd = self.hB.to(dev, non_blocking=True)
         if fmt == fp4.NVFP4:
-            gA = fp4.global_scale(Ad)
+            gA = torch.empty(1, dtype=torch.float32, device=dev)
             gB = torch.empty(1, dtype=torch.float32, device=dev)
             al = torch.empty(1, dtype=torch.float32, device=dev)
-            fp4.fp4_compute_global_scale_alpha(Bd, gB, gA, al)
+            fp4.fp4_compute_global_scales_pair(Ad, Bd, gA, gB, al)
         else:
             gA = gB = al = None
         pA, sA = _qbufs(fmt, n, n, dev)

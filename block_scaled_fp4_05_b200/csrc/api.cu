@@ -97,7 +97,7 @@ constexpr int64_t kMaxRowTiles = (int64_t)1 << 28;
 
 extern "C" {
 
-int fp4_abi_version(void) { return 3; }
+int fp4_abi_version(void) { return 4; }
 
 const char* fp4_last_error(void) { return fp4::g_last_error; }
 
@@ -166,6 +166,30 @@ fp4_status fp4_compute_global_scale_alpha(const void* in_bf16, int64_t rows, int
     return from_cuda(fp4::launch_global_scale(static_cast<const uint16_t*>(in_bf16), rows, cols, ld,
                                               gs_out, other_gs, alpha_out,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fp4_status fp4_compute_global_scales_pair(const void* a_bf16, int64_t rows_a, int64_t cols_a,
+                                          int64_t ld_a, const void* b_bf16, int64_t rows_b,
+                                          int64_t cols_b, int64_t ld_b, float* gs_a_out,
+                                          float* gs_b_out, float* alpha_out, fp4_stream_t stream)
+{
+    fp4::g_last_error[0] = 0;
+    if (rows_a < 0 || cols_a < 0 || rows_b < 0 || cols_b < 0 || gs_a_out == nullptr || gs_b_out == nullptr)
+        return FP4_ERR_INVALID_ARG;
+    if ((rows_a > 0 && cols_a > 0 && a_bf16 == nullptr) || (rows_b > 0 && cols_b > 0 && b_bf16 == nullptr))
+        return FP4_ERR_INVALID_ARG;
+    if (ld_a < cols_a || ld_b < cols_b) return FP4_ERR_INVALID_ARG;
+    if (cols_a % 8 != 0 || cols_b % 8 != 0) return FP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld_a % 8 != 0 || ld_b % 8 != 0 || !aligned16(a_bf16) || !aligned16(b_bf16) ||
+        (reinterpret_cast<uintptr_t>(gs_a_out) & 3u) || (reinterpret_cast<uintptr_t>(gs_b_out) & 3u) ||
+        (reinterpret_cast<uintptr_t>(alpha_out) & 3u))
+        return FP4_ERR_MISALIGNED;
+    fp4::DeviceInfo dev;
+    fp4_status st = require_device(&dev);
+    if (st != FP4_OK) return st;
+    return from_cuda(fp4::launch_global_scale_pair(
+        static_cast<const uint16_t*>(a_bf16), rows_a, cols_a, ld_a, static_cast<const uint16_t*>(b_bf16), rows_b,
+        cols_b, ld_b, gs_a_out, gs_b_out, alpha_out, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fp4_status fp4_quantize(fp4_format fmt, fp4_axis axis, const void* in_bf16, int64_t rows,

@@ -29,6 +29,11 @@ cudaError_t device_info(DeviceInfo* out);
 cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                                 float* gs_out, const float* other_gs, float* alpha_out,
                                 cudaStream_t s);
+// S_global of two tensors and alpha = gs_a * gs_b (alpha_out may be NULL) in
+// one launch.
+cudaError_t launch_global_scale_pair(const uint16_t* xa, int64_t rows_a, int64_t cols_a, int64_t ld_a,
+                                     const uint16_t* xb, int64_t rows_b, int64_t cols_b, int64_t ld_b,
+                                     float* gs_a, float* gs_b, float* alpha_out, cudaStream_t s);
 cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaStream_t s);
 cudaError_t launch_quantize_dynamic(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                                     uint8_t* packed, uint8_t* scales, float* gs_out,

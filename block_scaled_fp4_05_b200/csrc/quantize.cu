@@ -487,60 +487,82 @@ quantize_colwise_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t co
 // reduce into different slots.
 // ---------------------------------------------------------------------------
 struct GsSlot {
-    unsigned int amax;    // BF16 magnitude bits
-    unsigned int count;   // CTAs arrived
+    unsigned int amax[2];   // BF16 magnitude bits of each tensor
+    unsigned int count;     // CTAs arrived
+    unsigned int pad;
 };
 constexpr int kGsSlots = 1024;
 __device__ GsSlot g_gs_slots[kGsSlots];
 
-constexpr int kGsUnroll = 4;   // 16-byte loads in flight per thread
+constexpr int kGsUnroll = 8;   // 16-byte loads in flight per thread
 
-// Rows are split into segments of kThreads * kGsUnroll chunks (8 BF16 each);
-// the CTAs take segments in a grid-stride loop, so no per-load index
-// division is needed.  A contiguous matrix (ld == cols) is one long row.
+// One or two tensors per launch.  Each tensor's rows are split into segments
+// of kThreads * kGsUnroll chunks (8 BF16 each), segment s of the launch
+// belonging to tensor 1 from seg_begin1 on; the CTAs take segments in a
+// grid-stride loop, so no per-load index division is needed.  A contiguous
+// matrix (ld == cols) is one long row.
+struct GsArgs {
+    const uint16_t* x[2];
+    int64_t cpr[2], ld[2], spr[2];
+    int64_t seg_begin1, seg_total;
+    float* gs_out[2];
+    const float* other_gs;   // one tensor: alpha = gs * *other_gs (if alpha_out)
+    float* alpha_out;        // two tensors: alpha = gs[0] * gs[1] (if alpha_out)
+    int n;
+};
+
 __global__ void __launch_bounds__(kThreads)
-global_scale_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t cpr, int64_t ld,
-                    int64_t segs_per_row, GsSlot* __restrict__ slot, float* __restrict__ gs_out,
-                    const float* __restrict__ other_gs, float* __restrict__ alpha_out)
+global_scale_kernel(const __grid_constant__ GsArgs a, GsSlot* __restrict__ slot)
 {
     pdl_trigger();
-    const int64_t total = rows * segs_per_row;
-    uint32_t m = 0;
-    for (int64_t sidx = blockIdx.x; sidx < total; sidx += gridDim.x) {
-        const int64_t r = sidx / segs_per_row;
-        const int64_t c0 = (sidx - r * segs_per_row) * (kThreads * kGsUnroll) + threadIdx.x;
-        const uint4* row = reinterpret_cast<const uint4*>(x + r * ld);
+    uint32_t m[2] = {0u, 0u};
+    for (int64_t sidx = blockIdx.x; sidx < a.seg_total; sidx += gridDim.x) {
+        const int k = sidx >= a.seg_begin1 ? 1 : 0;
+        const int64_t ls = sidx - (k ? a.seg_begin1 : 0);
+        const int64_t r = ls / a.spr[k];
+        const int64_t c0 = (ls - r * a.spr[k]) * (kThreads * kGsUnroll) + threadIdx.x;
+        const uint4* row = reinterpret_cast<const uint4*>(a.x[k] + r * a.ld[k]);
         uint4 v[kGsUnroll];
 #pragma unroll
         for (int u = 0; u < kGsUnroll; ++u) {
             const int64_t c = c0 + u * kThreads;
-            v[u] = c < cpr ? ld_stream(row + c) : make_uint4(0u, 0u, 0u, 0u);
+            v[u] = c < a.cpr[k] ? ld_stream(row + c) : make_uint4(0u, 0u, 0u, 0u);
         }
+        uint32_t mm = 0;
 #pragma unroll
-        for (int u = 0; u < kGsUnroll; ++u) m = max(m, absmax8(v[u]));
+        for (int u = 0; u < kGsUnroll; ++u) mm = max(mm, absmax8(v[u]));
+        m[k] = max(m[k], mm);
     }
+    __shared__ uint32_t s_m[2][kThreads / 32];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    __shared__ uint32_t s_m[kThreads / 32];
-    if ((threadIdx.x & 31) == 0) s_m[threadIdx.x >> 5] = m;
+    for (int k = 0; k < 2; ++k) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m[k] = max(m[k], __shfl_xor_sync(0xFFFFFFFFu, m[k], o));
+        if ((threadIdx.x & 31) == 0) s_m[k][threadIdx.x >> 5] = m[k];
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
-        uint32_t b = 0;
-        for (int w = 0; w < kThreads / 32; ++w) b = max(b, s_m[w]);
-        if (b) atomicMax(&slot->amax, b);
-        // release: this CTA's maximum is visible before its arrival counts;
-        // acquire: the last arriver sees every other CTA's maximum
+        for (int k = 0; k < a.n; ++k) {
+            uint32_t b = 0;
+            for (int w = 0; w < kThreads / 32; ++w) b = max(b, s_m[k][w]);
+            if (b) atomicMax(&slot->amax[k], b);
+        }
+        // release: this CTA's maxima are visible before its arrival counts;
+        // acquire: the last arriver sees every other CTA's maxima
         unsigned int old;
         asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
                      : "=r"(old) : "l"(&slot->count) : "memory");
         if (old == gridDim.x - 1) {
-            unsigned int bits;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(&slot->amax) : "memory");
-            const float amax = __uint_as_float(bits << 16);
-            const float gs = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-            *gs_out = gs;
-            if (alpha_out) *alpha_out = __fmul_rn(gs, *other_gs);
-            slot->amax = 0u;
+            float gs[2] = {1.0f, 1.0f};
+            for (int k = 0; k < a.n; ++k) {
+                unsigned int bits;
+                asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(bits) : "l"(&slot->amax[k]) : "memory");
+                const float amax = __uint_as_float(bits << 16);
+                gs[k] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                *a.gs_out[k] = gs[k];
+                slot->amax[k] = 0u;
+            }
+            if (a.alpha_out) *a.alpha_out = __fmul_rn(gs[0], a.n == 2 ? gs[1] : *a.other_gs);
             slot->count = 0u;
         }
     }
@@ -585,9 +607,22 @@ cudaError_t launch_alpha(const float* gsA, const float* gsB, float* alpha, cudaS
     return cudaGetLastError();
 }
 
-cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                                float* gs_out, const float* other_gs, float* alpha_out,
-                                cudaStream_t s)
+// Segments of one tensor: a contiguous matrix (ld == cols) is reduced as one
+// row.
+static void gs_tensor(GsArgs& a, int k, const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                      float* gs_out, int64_t* nseg)
+{
+    const bool flat = ld == cols;
+    const int64_t r = flat ? 1 : rows;
+    a.x[k] = x;
+    a.cpr[k] = flat ? rows * cols / 8 : cols / 8;
+    a.ld[k] = ld;
+    a.spr[k] = (a.cpr[k] + kThreads * kGsUnroll - 1) / (kThreads * kGsUnroll);
+    a.gs_out[k] = gs_out;
+    *nseg = (rows == 0 || cols == 0) ? 0 : r * a.spr[k];
+}
+
+static cudaError_t launch_gs(GsArgs& a, int64_t seg0, int64_t seg1, cudaStream_t s)
 {
     static unsigned int next_slot = 0;   // ring position (atomic: calls from several threads)
     DeviceInfo dev;
@@ -597,18 +632,40 @@ cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, i
     e = gs_slots(&slots);
     if (e != cudaSuccess) return e;
     const unsigned int k = __atomic_fetch_add(&next_slot, 1u, __ATOMIC_RELAXED) % kGsSlots;
-    // a contiguous matrix is reduced as one row
-    const bool flat = ld == cols;
-    const int64_t r = flat ? 1 : rows;
-    const int64_t cpr = flat ? rows * cols / 8 : cols / 8;
-    const int64_t spr = (cpr + kThreads * kGsUnroll - 1) / (kThreads * kGsUnroll);
-    int64_t grid = r * spr;
+    a.seg_begin1 = seg0;
+    a.seg_total = seg0 + seg1;
+    int64_t grid = a.seg_total;
     const int64_t cap = (int64_t)dev.sm_count * 8;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    global_scale_kernel<<<(unsigned)grid, kThreads, 0, s>>>(x, r, cpr, ld, spr, slots + k, gs_out,
-                                                            other_gs, alpha_out);
+    global_scale_kernel<<<(unsigned)grid, kThreads, 0, s>>>(a, slots + k);
     return cudaGetLastError();
+}
+
+cudaError_t launch_global_scale(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                float* gs_out, const float* other_gs, float* alpha_out,
+                                cudaStream_t s)
+{
+    GsArgs a = {};
+    int64_t n0 = 0;
+    gs_tensor(a, 0, x, rows, cols, ld, gs_out, &n0);
+    a.n = 1;
+    a.other_gs = other_gs;
+    a.alpha_out = alpha_out;
+    return launch_gs(a, n0, 0, s);
+}
+
+cudaError_t launch_global_scale_pair(const uint16_t* xa, int64_t rows_a, int64_t cols_a, int64_t ld_a,
+                                     const uint16_t* xb, int64_t rows_b, int64_t cols_b, int64_t ld_b,
+                                     float* gs_a, float* gs_b, float* alpha_out, cudaStream_t s)
+{
+    GsArgs a = {};
+    int64_t n0 = 0, n1 = 0;
+    gs_tensor(a, 0, xa, rows_a, cols_a, ld_a, gs_a, &n0);
+    gs_tensor(a, 1, xb, rows_b, cols_b, ld_b, gs_b, &n1);
+    a.n = 2;
+    a.alpha_out = alpha_out;
+    return launch_gs(a, n0, n1, s);
 }
 
 namespace {

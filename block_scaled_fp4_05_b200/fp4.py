@@ -62,6 +62,8 @@ def lib():
         L.fp4_compute_global_scale.argtypes = [P, i64, i64, i64, P, st]
         L.fp4_compute_global_scale_alpha.restype = c.c_int
         L.fp4_compute_global_scale_alpha.argtypes = [P, i64, i64, i64, P, P, P, st]
+        L.fp4_compute_global_scales_pair.restype = c.c_int
+        L.fp4_compute_global_scales_pair.argtypes = [P, i64, i64, i64, P, i64, i64, i64, P, P, P, st]
         L.fp4_quantize.restype = c.c_int
         L.fp4_quantize.argtypes = [c.c_int, c.c_int, P, i64, i64, i64, P, P, P, st]
         L.fp4_gemm_grouped.restype = c.c_int
@@ -123,6 +125,8 @@ def _dptr(t, what):
 
 
 def _ld(t):
+    if t.dim() == 2 and t.numel() == 0:
+        return t.shape[1]            # an empty matrix: any stride torch reports
     if t.dim() != 2 or t.stride(1) != 1:
         raise ValueError("expected a 2-D tensor with unit column stride")
     return t.stride(0)
@@ -160,6 +164,16 @@ def fp4_compute_global_scale_alpha(x, gs_out, other_gs, alpha_out, stream=None):
                                                 _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"),
                                                 _dptr(alpha_out, "alpha_out"), _stream(stream)),
            "fp4_compute_global_scale_alpha")
+
+
+def fp4_compute_global_scales_pair(a, b, gs_a_out, gs_b_out, alpha_out=None, stream=None):
+    """S_global of a and of b and (if alpha_out) alpha = gs_a * gs_b, one launch."""
+    assert a.dtype == torch.bfloat16 and b.dtype == torch.bfloat16
+    _check(lib().fp4_compute_global_scales_pair(_dptr(a, "a"), a.shape[0], a.shape[1], _ld(a),
+                                                _dptr(b, "b"), b.shape[0], b.shape[1], _ld(b),
+                                                _dptr(gs_a_out, "gs_a_out"), _dptr(gs_b_out, "gs_b_out"),
+                                                _dptr(alpha_out, "alpha_out"), _stream(stream)),
+           "fp4_compute_global_scales_pair")
 
 
 def fp4_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):
@@ -381,6 +395,12 @@ def bind_global_scale_alpha(x, gs_out, other_gs, alpha_out, stream=None):
     return BoundCall("fp4_compute_global_scale_alpha", _dptr(x, "x"), x.shape[0], x.shape[1], _ld(x),
                      _dptr(gs_out, "gs_out"), _dptr(other_gs, "other_gs"), _dptr(alpha_out, "alpha_out"),
                      _stream(stream))
+
+
+def bind_global_scales_pair(a, b, gs_a_out, gs_b_out, alpha_out=None, stream=None):
+    return BoundCall("fp4_compute_global_scales_pair", _dptr(a, "a"), a.shape[0], a.shape[1], _ld(a),
+                     _dptr(b, "b"), b.shape[0], b.shape[1], _ld(b), _dptr(gs_a_out, "gs_a_out"),
+                     _dptr(gs_b_out, "gs_b_out"), _dptr(alpha_out, "alpha_out"), _stream(stream))
 
 
 def bind_quantize(fmt, axis, x, packed_out, scales_out, global_scale=None, stream=None):

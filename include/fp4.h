@@ -152,6 +152,23 @@ fp4_status fp4_compute_global_scale_alpha(const void* in_bf16, int64_t rows, int
                                           float* alpha_out, fp4_stream_t stream);
 
 /*
+ * S_global of both operands of an NVFP4 GEMM and alpha = gs_a * gs_b, in one
+ * launch (the CTAs of that launch reduce the rows of either tensor; the last
+ * to finish writes both scales and alpha): each value equal to what
+ * fp4_compute_global_scale and fp4_alpha_from_global_scales give.  Same
+ * reading of [NVFP4-Arch] "1. The Dual-Level Mathematical Formulation" as
+ * above, for the two tensors whose product the GEMM forms.
+ *   a_bf16, b_bf16 : device, rows x cols each, leading dimension ld_*
+ *   gs_a_out, gs_b_out : device floats, written
+ *   alpha_out : device float, or NULL
+ * Requires cols_* % 8 == 0; an empty tensor gets S_global = 1.
+ */
+fp4_status fp4_compute_global_scales_pair(const void* a_bf16, int64_t rows_a, int64_t cols_a,
+                                          int64_t ld_a, const void* b_bf16, int64_t rows_b,
+                                          int64_t cols_b, int64_t ld_b, float* gs_a_out,
+                                          float* gs_b_out, float* alpha_out, fp4_stream_t stream);
+
+/*
  * Block quantization BF16 -> E2M1 codes + one scale per block.
  * [NVFP4-Arch] "1. The Dual-Level Mathematical Formulation" (S_block,j,
  * q_i = Quantize_E2M1(x_i / (S_global * S_block,j))) and the emulation script

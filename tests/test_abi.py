@@ -13,7 +13,7 @@ def test_library_exports_every_declared_symbol():
     assert len(names) >= 12
     for n in names:
         assert hasattr(L, n), n
-    assert L.fp4_abi_version() == 3
+    assert L.fp4_abi_version() == 4
 
 
 def test_status_strings():
@@ -173,6 +173,22 @@ def test_global_scale_alpha_host_checks_without_gpu():
     assert f(A16, 4, 8, 8, A16, A16, P((1 << 20) + 2), None) == 3   # misaligned alpha
     if not torch.cuda.is_available():
         assert f(A16, 4, 8, 8, A16, A16, A16, None) == 6
+
+
+def test_global_scales_pair_host_checks_without_gpu():
+    import torch
+    L = fp4.lib()
+    f = L.fp4_compute_global_scales_pair
+    # (a, rows_a, cols_a, ld_a, b, rows_b, cols_b, ld_b, gs_a, gs_b, alpha, stream)
+    assert f(A16, 4, 8, 8, A16, 4, 8, 8, None, A16, A16, None) == 1      # no gs_a_out
+    assert f(A16, 4, 8, 8, A16, 4, 8, 8, A16, None, A16, None) == 1      # no gs_b_out
+    assert f(A16, 4, 8, 8, None, 4, 8, 8, A16, A16, A16, None) == 1      # no b
+    assert f(A16, 4, 8, 8, A16, 4, 8, 4, A16, A16, A16, None) == 1       # ld_b < cols_b
+    assert f(A16, 4, 12, 12, A16, 4, 8, 8, A16, A16, A16, None) == 2     # cols_a % 8
+    assert f(A16, 4, 8, 8, A1, 4, 8, 8, A16, A16, A16, None) == 3        # misaligned b
+    assert f(A16, 4, 8, 8, A16, 4, 8, 8, A16, A16, P((1 << 20) + 2), None) == 3   # misaligned alpha
+    if not torch.cuda.is_available():
+        assert f(A16, 4, 8, 8, A16, 4, 8, 8, A16, A16, None, None) == 6
 
 
 def test_decode_dynamic_host_checks_without_gpu():

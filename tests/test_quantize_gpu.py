@@ -144,6 +144,29 @@ def test_global_scale_alpha_one_launch(orc):
     assert np.float32(al.item()) == np.float32(g) * np.float32(0.0371)
 
 
+@pytest.mark.parametrize("shapes", [((100, 256, 264), (64, 512, 512)), ((4096, 4096, 4096), (4096, 4096, 4096)),
+                                    ((0, 64, 64), (33, 72, 80)), ((2048, 8192, 8192), (1, 8, 8))])
+def test_global_scales_pair_one_launch(orc, shapes):
+    # both operands' S_global and alpha from one launch, identical to the
+    # single-tensor calls and to the oracle; strided views, an empty tensor
+    # (S_global = 1) and tensors of very different sizes
+    (ra, ca, la), (rb, cb, lb) = shapes
+    xa = synth.normal_bf16(ra, ca, seed=31, outlier_factor=30.0) if ra else np.zeros((0, ca), np.uint16)
+    xb = synth.normal_bf16(rb, cb, seed=31, tensor_id=1, outlier_factor=7.0)
+    da, db = [to_dev_bf16(np.pad(x, ((0, 0), (0, l - x.shape[1])))) for x, l in ((xa, la), (xb, lb))]
+    out = torch.zeros(3, dtype=torch.float32, device="cuda")
+    fp4.fp4_compute_global_scales_pair(da[:, :ca], db[:, :cb], out[0:1], out[1:2], out[2:3])
+    torch.cuda.synchronize()
+    ga = np.float32(orc.global_scale(xa)) if ra else np.float32(1.0)
+    gb = np.float32(orc.global_scale(xb))
+    got = out.cpu().numpy()
+    assert got[0] == ga and got[1] == gb and got[2] == ga * gb
+    one = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_compute_global_scale(db[:, :cb], one)
+    torch.cuda.synchronize()
+    assert one.item() == got[1]
+
+
 def test_global_scale_slot_ring_wraps(orc):
     # more calls than reduction slots, alternating two tensors: every call
     # leaves its slot zeroed, so the second use of each slot is exact again
