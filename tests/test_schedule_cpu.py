@@ -89,3 +89,70 @@ def test_headline_decode_shape():
     assert (G, sk, ms) == (148, 76, 2)
     loads = [sum(ke - kb for _, kb, ke, _ in segments(c, G, sk, 32, 224)) for c in range(G)]
     assert min(loads) == 48 and max(loads) == 49
+
+
+# ---------------------------------------------------------------------------
+# The prefill (pair) kernel's work items, restated: tiles dealt to the CTA
+# pairs round-robin; when the last wave has R < pairs tiles and 2R <= pairs,
+# those R tiles run as 2R column halves (launch_pair and locate() in
+# csrc/gemm.cu).
+# ---------------------------------------------------------------------------
+def pair_launch(tiles, max_pairs, single_problem=True):
+    rem = tiles % max_pairs
+    split = single_problem and rem > 0 and 2 * rem <= max_pairs
+    split_from = tiles - rem if split else tiles
+    items = tiles + (rem if split else 0)
+    npairs = min(items, max_pairs)
+    return split_from, items, npairs
+
+
+def pair_locate(t, split_from):
+    if t < split_from:
+        return t, 0
+    return split_from + ((t - split_from) >> 1), 1 + ((t - split_from) & 1)
+
+
+@pytest.mark.parametrize("tiles", [1, 2, 5, 33, 37, 38, 73, 74, 75, 88, 110, 111, 112, 148, 256, 1024, 3584])
+@pytest.mark.parametrize("max_pairs", [74, 66, 1])
+def test_pair_items_cover_every_tile_once(tiles, max_pairs):
+    split_from, items, npairs = pair_launch(tiles, max_pairs)
+    seen = {}
+    per_pair = []
+    for pair in range(npairs):
+        mine = list(range(pair, items, npairs))
+        per_pair.append(mine)
+        for t in mine:
+            ft, nh = pair_locate(t, split_from)
+            assert 0 <= ft < tiles
+            key = (ft, nh)
+            assert key not in seen, "work item computed twice"
+            seen[key] = pair
+    for ft in range(tiles):
+        whole = (ft, 0) in seen
+        halves = (ft, 1) in seen and (ft, 2) in seen
+        assert whole != halves, "tile %d: whole=%s halves=%s" % (ft, whole, halves)
+        assert ((ft, 1) in seen) == ((ft, 2) in seen)
+        if halves:
+            assert seen[(ft, 1)] != seen[(ft, 2)], "both halves on one pair"
+            assert ft >= tiles - tiles % max_pairs, "only the last wave is split"
+    # every pair runs the same number of whole tiles, at most one half tile,
+    # and the half tiles come last
+    full_rounds = split_from // npairs if npairs else 0
+    for mine in per_pair:
+        halves = [t for t in mine if t >= split_from]
+        assert len(halves) <= 1
+        assert len(mine) - len(halves) in (full_rounds, full_rounds + (1 if split_from % npairs else 0))
+        assert all(t >= split_from for t in mine[len(mine) - len(halves):])
+
+
+def test_pair_split_cases():
+    # 4096^2 (16 x 16 tiles) on 74 pairs: 34 leftover tiles -> 68 halves
+    assert pair_launch(256, 74) == (222, 290, 74)
+    # 8192 x 28672: 32 x 112 = 3584 tiles, 32 left -> split
+    assert pair_launch(3584, 74)[0] == 3552
+    # 8192 x 8192: 1024 tiles, 62 left > 37 -> no split
+    assert pair_launch(1024, 74) == (1024, 1024, 74)
+    # fewer tiles than half the pairs: every tile split, one half per pair
+    assert pair_launch(5, 74) == (0, 10, 10)
+    # grouped launches never split
+    assert pair_launch(256, 74, single_problem=False)[0] == 256
