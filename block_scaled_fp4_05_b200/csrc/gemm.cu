@@ -1385,8 +1385,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
                     if (leader)
                         mbar_arrive_expect_tx(B_FULL(stage), 2u * (A_BYTES + C::B_BYTES));
                     const uint32_t full_leader = map_to_rank(B_FULL(stage), 0);
-                    tma_load_2d_pair(&args.a[g], full_leader, st, ks * BK_BYTES, ya);
-                    tma_load_2d_pair(&args.b[g], full_leader, st + C::OFF_B, ks * BK_BYTES, yb);
+                    // the scale chunks first: they land before the operand tiles, so
+                    // their staging into TMEM stays off the slot's critical path
                     mbar_arrive_expect_tx(B_SFFULL(stage), sf_bytes * ((has_sfa ? 1 : 0) + nbh));
                     if (has_sfa)
                         bulk_load(st + C::OFF_SFA, sfa_row + ct0 * SF_CHUNK, sf_bytes, B_SFFULL(stage));
@@ -1395,6 +1395,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
                     if (nbh > 1)
                         bulk_load(st + C::OFF_SFB + C::SFA_STAGE, sfb_row + sf_row_bytes + ct0 * SF_CHUNK,
                                   sf_bytes, B_SFFULL(stage));
+                    tma_load_2d_pair(&args.a[g], full_leader, st, ks * BK_BYTES, ya);
+                    tma_load_2d_pair(&args.b[g], full_leader, st + C::OFF_B, ks * BK_BYTES, yb);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -1541,7 +1543,8 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
             tmem_ld32(trow + 96, rb);
             convert(ra, 2);
             tmem_wait_ld(rb);
-            convert(rb, 3);
+            // every column is in registers: hand the accumulator back before
+            // converting the last chunk
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -1550,6 +1553,7 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
                 else
                     mbar_arrive_cluster_relaxed(acc_empty_leader);
             }
+            convert(rb, 3);
             // D through shared memory: the warp's 32 rows x 32 columns at a
             // time go to its staging block (64-byte rows; 16-byte chunk j of
             // row r at chunk j ^ ((r >> 1) & 3), the 64-byte swizzle), then
