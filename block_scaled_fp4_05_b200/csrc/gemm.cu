@@ -28,6 +28,10 @@
 //               tcgen05.st, so that the tensor pipe only runs MMAs (a
 //               tcgen05.cp of a 512-byte chunk occupies the tensor pipe for
 //               about half the time of a 128x256x64 MMA).
+//   warps 10-13 (the decode tile, N = 16, only) when the activation arrives
+//               as BF16: each forms the NVFP4 codes and scales of every
+//               fourth stage's activation slice straight into that stage's
+//               shared-memory slot (otherwise they idle).
 // Every mbarrier wait is bounded by %globaltimer; on expiry the CTA sets the
 // library's device error word, stops issuing work, drains what it already
 // issued, frees its tensor memory and returns (no trap).
