@@ -127,3 +127,33 @@ def test_w4a4_vs_w4a16_vs_naive_per_tensor(orc, MNK, record_property):
     # a single per-tensor scale collapses the non-outlier values
     assert snr["w4a16_nvfp4_weights"] > snr["w4a4_nvfp4"] > snr["w4a4_mxfp4"] > snr["naive_per_tensor_fp4"]
     assert snr["naive_per_tensor_fp4"] < 10.0 < snr["w4a4_mxfp4"]
+
+
+def test_square_4096_error_nv_below_mx(record_property):
+    # The 4096^3 inputs (outlier channels in A), quantized on the GPU in both
+    # formats and multiplied by the GPU GEMM: relative Frobenius error and SNR
+    # of D against the FP64 product of the original BF16 inputs (computed on
+    # the GPU in FP64).  NVFP4's 16-element blocks with E4M3 scales must give
+    # the smaller error (an invariant of the formats, not a pinned value).
+    A, B = synth.square(4096)
+    Ad, Bd = to_dev_bf16(A), to_dev_bf16(B)
+    ref = Ad.double() @ Bd.double().T
+    err = {}
+    for fmt, name in ((fp4.NVFP4, "nvfp4"), (fp4.MXFP4, "mxfp4")):
+        gA = fp4.global_scale(Ad) if fmt == fp4.NVFP4 else None
+        gB = fp4.global_scale(Bd) if fmt == fp4.NVFP4 else None
+        pA, sA = fp4.quantize(Ad, fmt, fp4.ROWWISE, gA)
+        pB, sB = fp4.quantize(Bd, fmt, fp4.ROWWISE, gB)
+        alpha = gA * gB if fmt == fp4.NVFP4 else None
+        D = fp4.gemm(fmt, pA, sA, pB, sB, 4096, alpha=alpha, kernel=fp4.GEMM_PREFILL)
+        torch.cuda.synchronize()
+        assert fp4.fp4_get_device_status() == 0
+        diff = D.double() - ref
+        rel = float(torch.linalg.norm(diff) / torch.linalg.norm(ref))
+        err[name] = (rel, -20.0 * np.log10(rel))
+        record_property("rel_fro_" + name, rel)
+    print("4096^3 relative Frobenius error / SNR: NVFP4 %.4f / %.2f dB, MXFP4 %.4f / %.2f dB" % (
+        err["nvfp4"][0], err["nvfp4"][1], err["mxfp4"][0], err["mxfp4"][1]))
+    assert err["nvfp4"][0] < err["mxfp4"][0]
+    assert err["nvfp4"][0] < 0.2 and err["mxfp4"][0] < 0.3
+
