@@ -61,8 +61,9 @@ def test_tiny_config(orc, fmt):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
+# K = 64: a single MMA per tile (NVFP4, P1E8); (130, 72, 64) also a ragged half tile
 @pytest.mark.parametrize("MNK", [(1, 8, 128), (3, 24, 256), (129, 136, 384), (200, 264, 640),
-                                 (300, 520, 1024), (128, 256, 2048), (257, 512, 128)])
+                                 (300, 520, 1024), (128, 256, 2048), (257, 512, 128), (130, 72, 64)])
 def test_prefill_ragged_shapes(orc, fmt, MNK):
     M, N, K = MNK
     if K % (128 if fmt == fp4.MXFP4 else 64):
@@ -79,7 +80,7 @@ def test_prefill_ragged_shapes(orc, fmt, MNK):
 # (16, 38400, 1024) and (9, 38400, 1088): more weight tiles than SMs, so the
 # decode schedule runs stream-K tiles and then whole tiles; 1088 adds a K tail
 @pytest.mark.parametrize("MNK", [(1, 256, 512), (4, 1000, 1024), (16, 1024, 8192), (7, 136, 384),
-                                 (16, 38400, 1024), (9, 38400, 1088)])
+                                 (16, 38400, 1024), (9, 38400, 1088), (5, 200, 64), (12, 520, 192)])
 def test_decode_kernel_shapes(orc, fmt, MNK):
     M, N, K = MNK
     if K % (128 if fmt == fp4.MXFP4 else 64):
