@@ -40,7 +40,8 @@ def test_f64_to_bf16_helper_against_torch():
 
 
 @pytest.mark.parametrize("fmt", [fp4.NVFP4, fp4.MXFP4, fp4.P1E8])
-@pytest.mark.parametrize("shape", [(1, 512), (200, 1024), (129, 8192)])
+# (33, 2176): a row is one whole 2048-code warp task plus a 128-code tail
+@pytest.mark.parametrize("shape", [(1, 512), (200, 1024), (129, 8192), (33, 2176)])
 def test_dequantize_matches_oracle(orc, fmt, shape):
     rows, K = shape
     x = synth.normal_bf16(rows, K, seed=61, outlier_factor=100.0, zero_frac=0.02)
