@@ -124,6 +124,7 @@ struct Params {
     int32_t units;             // stream-K: sk_tiles * ks_total
     int32_t sk_tiles;          // stream-K: tiles split over the CTAs; the rest run whole
     int32_t a_static;          // A side not written by the previous kernel: prefetch it
+    int32_t raster_gm;         // pair kernel: M tiles per group of the tile order
     int32_t max_seg;           // stream-K: partial slots per CTA
     const float* alpha;
     uint16_t* D;
@@ -1081,6 +1082,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // CTAs meet at a final cluster barrier before the pair frees its TMEM.
 // ------------------------------------------------------------------------
 constexpr int PAIR_BN = 256;                 // N of the pair tile
+constexpr int64_t kRasterGroupBytes = int64_t(32) << 20;   // A bytes per raster group
 constexpr int PAIR_BHALF = PAIR_BN / 2;      // B rows staged by each CTA
 constexpr int kPairThreads = 448;            // 14 warps, roles above
 constexpr int kEpiWarps = 8;
@@ -1344,8 +1346,18 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
         if (NG > 1)
             while (g + 1 < args.n && ft >= args.tile_begin[g + 1]) ++g;
         const int lt = ft - args.tile_begin[g];
-        tm = lt % args.p[g].tiles_m;
-        tn = lt / args.p[g].tiles_m;
+        // grouped raster: raster_gm consecutive M tiles sweep the N tiles
+        // together (M fastest inside a group), so that the A row blocks of a
+        // group stay in L2 while the B row blocks stream past them once per
+        // group (raster_gm = tiles_m: plain M-fastest order)
+        const int tiles_m = args.p[g].tiles_m;
+        const int rg = args.p[g].raster_gm;
+        const int span = rg * args.p[g].tiles_n;
+        const int grp = lt / span, in = lt - grp * span;
+        const int m0 = grp * rg;
+        const int gm = min(tiles_m - m0, rg);
+        tm = m0 + in % gm;
+        tn = in / gm;
     };
 
     if (warp == 0) {
@@ -1878,6 +1890,7 @@ static void fill_common(Params& p, const GemmArgs& a, int64_t rows_a, int64_t ro
     p.sk_tiles = 0;
     p.a_static = 0;
     p.max_seg = 0;
+    p.raster_gm = 1;
 }
 
 template <int STAGES, int FMT, int NG>
@@ -1934,6 +1947,14 @@ bool fill_pair_problem(PairArgs<NG>& args, int g, const GemmArgs& a)
     fill_common(p, a, a.M, a.N, a.sA, a.sB);
     p.tiles_m = (int32_t)((a.M + 255) / 256);
     p.tiles_n = (int32_t)((a.N + PAIR_BN - 1) / PAIR_BN);
+    // tile order: plain M-fastest when all of A (codes and scales) fits in
+    // about half of the L2 cache, else groups of M tiles whose A rows fit in
+    // kRasterGroupBytes, so that B streams past each group once
+    const int64_t a_tile_bytes = 256 * (a.K / 2 + a.K / block_size(a.fmt));
+    int64_t rg = p.tiles_m;
+    if (a_tile_bytes * p.tiles_m > (int64_t)(64 << 20))
+        rg = (kRasterGroupBytes + a_tile_bytes / 2) / a_tile_bytes;
+    p.raster_gm = (int32_t)(rg < 1 ? 1 : (rg > p.tiles_m ? p.tiles_m : rg));
     args.tile_begin[g + 1] = args.tile_begin[g] + p.tiles_m * p.tiles_n;
     return true;
 }

@@ -156,3 +156,50 @@ def test_pair_split_cases():
     assert pair_launch(5, 74) == (0, 10, 10)
     # grouped launches never split
     assert pair_launch(256, 74, single_problem=False)[0] == 256
+
+
+# The pair kernel's tile order (locate() in csrc/gemm.cu): groups of rg
+# consecutive M tiles sweep the N tiles together, M fastest inside a group;
+# rg is chosen on the host (fill_pair_problem): all M tiles when A fits in
+# 64 MB, else as many as put about 32 MB of A rows in a group.
+def raster(lt, tiles_m, tiles_n, rg):
+    span = rg * tiles_n
+    grp, i = divmod(lt, span)
+    m0 = grp * rg
+    gm = min(tiles_m - m0, rg)
+    return m0 + i % gm, i // gm
+
+
+def raster_group(M, K, block):
+    tiles_m = (M + 255) // 256
+    a_tile = 256 * (K // 2 + K // block)
+    rg = tiles_m
+    if a_tile * tiles_m > (64 << 20):
+        rg = ((32 << 20) + a_tile // 2) // a_tile
+    return max(1, min(tiles_m, rg))
+
+
+@pytest.mark.parametrize("tiles_m,tiles_n", [(1, 1), (1, 7), (5, 1), (16, 16), (32, 112), (32, 32), (13, 9), (33, 5)])
+@pytest.mark.parametrize("rg", [1, 3, 8, 16, 32, 64])
+def test_raster_is_a_bijection(tiles_m, tiles_n, rg):
+    rg = min(rg, tiles_m)
+    seen = set()
+    for lt in range(tiles_m * tiles_n):
+        tm, tn = raster(lt, tiles_m, tiles_n, rg)
+        assert 0 <= tm < tiles_m and 0 <= tn < tiles_n
+        seen.add((tm, tn))
+    assert len(seen) == tiles_m * tiles_n
+    if rg == tiles_m:   # one group: the plain M-fastest order
+        assert all(raster(lt, tiles_m, tiles_n, rg) == (lt % tiles_m, lt // tiles_m)
+                   for lt in range(tiles_m * tiles_n))
+
+
+def test_raster_groups_for_the_bench_shapes():
+    # 8192 x 28672 x 8192 and 4096^3: A fits in L2, the order stays M-fastest
+    assert raster_group(8192, 8192, 16) == 32
+    assert raster_group(4096, 4096, 32) == 16
+    # 8192 x 8192 x 28672: 4.1 MB of A per M tile (132 MB in all), 8 per group
+    assert raster_group(8192, 28672, 16) == 8
+    # a wave of 74 consecutive tiles then touches at most 8 M tiles
+    tms = {raster(lt, 32, 32, 8)[0] for lt in range(74)}
+    assert len(tms) <= 8
