@@ -579,11 +579,14 @@ class PrefillWorkload(Workload):
         t_step = ((t1 - t0) + (t2 - t1) * nbm / len(qa) + (t3 - t2) * (nbm * nbn) / tiles)
         return t_step, t3 - t0
 
-    def calibrate(self, orc, budget_s, max_tiles=64):
-        """Tile count whose sample takes about budget_s seconds (4..max_tiles)."""
-        _, spent = self.oracle_sample(orc, 2, seed=1)
-        per_tile = max(spent / 2, 1e-3)
-        return int(max(4, min(max_tiles, budget_s / per_tile)))
+    def calibrate(self, orc, budget_s, max_tiles=4096):
+        """Tile count whose sample takes about budget_s seconds (4..max_tiles):
+        the fixed part (S_global of the whole activation) and the cost of one
+        more tile come from two short probes."""
+        _, fixed = self.oracle_sample(orc, 2, seed=1)
+        _, spent = self.oracle_sample(orc, 18, seed=2)
+        per_tile = max((spent - fixed) / 16, 1e-3)
+        return int(max(4, min(max_tiles, (budget_s - fixed) / per_tile)))
 
     def sample_note(self, tiles):
         return ("S_global of the whole %dx%d activation, quantization of the sampled 128-row "
