@@ -515,7 +515,7 @@ __global__ void __launch_bounds__(kThreads)
 global_scale_kernel(const __grid_constant__ GsArgs a, GsSlot* __restrict__ slot)
 {
     pdl_trigger();
-    uint32_t m[2] = {0u, 0u};
+    uint32_t m0 = 0u, m1 = 0u;   // the two tensors' maxima (registers, not an indexed array)
     for (int64_t sidx = blockIdx.x; sidx < a.seg_total; sidx += gridDim.x) {
         const int k = sidx >= a.seg_begin1 ? 1 : 0;
         const int64_t ls = sidx - (k ? a.seg_begin1 : 0);
@@ -531,8 +531,9 @@ global_scale_kernel(const __grid_constant__ GsArgs a, GsSlot* __restrict__ slot)
         uint32_t mm = 0;
 #pragma unroll
         for (int u = 0; u < kGsUnroll; ++u) mm = max(mm, absmax8(v[u]));
-        m[k] = max(m[k], mm);
+        if (k) m1 = max(m1, mm); else m0 = max(m0, mm);
     }
+    uint32_t m[2] = {m0, m1};
     __shared__ uint32_t s_m[2][kThreads / 32];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
@@ -622,6 +623,28 @@ static void gs_tensor(GsArgs& a, int k, const uint16_t* x, int64_t rows, int64_t
     *nseg = (rows == 0 || cols == 0) ? 0 : r * a.spr[k];
 }
 
+// Resident CTAs per SM of the S_global kernel (per device, looked up once).
+static int global_scale_blocks_per_sm()
+{
+    static std::mutex mu;
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 4;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 64 && cache[dev]) return cache[dev];
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, global_scale_kernel, kThreads, 0) != cudaSuccess ||
+        nb < 1) {
+        cudaGetLastError();
+        nb = 4;
+    }
+    if (dev < 64) cache[dev] = nb;
+    return nb;
+}
+
 static cudaError_t launch_gs(GsArgs& a, int64_t seg0, int64_t seg1, cudaStream_t s)
 {
     static unsigned int next_slot = 0;   // ring position (atomic: calls from several threads)
@@ -635,7 +658,8 @@ static cudaError_t launch_gs(GsArgs& a, int64_t seg0, int64_t seg1, cudaStream_t
     a.seg_begin1 = seg0;
     a.seg_total = seg0 + seg1;
     int64_t grid = a.seg_total;
-    const int64_t cap = (int64_t)dev.sm_count * 8;
+    // one wave: every CTA resident from the start, segments taken grid-stride
+    const int64_t cap = (int64_t)dev.sm_count * global_scale_blocks_per_sm();
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     global_scale_kernel<<<(unsigned)grid, kThreads, 0, s>>>(a, slots + k);

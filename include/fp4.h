@@ -247,8 +247,8 @@ fp4_status fp4_quantize_batch(fp4_format fmt, int n, const fp4_quantize_desc* de
  * fp4_alpha_from_global_scales with the other operand's scale).  Results are
  * identical to those three calls.  One cluster of 16 CTAs (8 where the device
  * cannot place 16) holds the tensor in registers between the amax and the
- * quantization; a tensor above that capacity (65536 16-byte chunks, i.e.
- * 1 MiB of BF16, with 16 CTAs) is handled inside the same call by two
+ * quantization; a tensor above that capacity (32768 16-byte chunks, i.e.
+ * 512 KiB of BF16, with 16 CTAs) is handled inside the same call by two
  * launches: S_global and alpha (as fp4_compute_global_scale_alpha), then the
  * rowwise quantizer, which visits the tensor's tiles last to first so that
  * the rows the first pass read last are still in L2.

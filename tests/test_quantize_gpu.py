@@ -235,11 +235,12 @@ def test_full_size_sweep_sampled_p1e8(orc, axis):
 
 
 @pytest.mark.parametrize("shape", [(1, 8192), (4, 8192), (16, 8192), (16, 512), (3, 64), (1, 64),
-                                   (200, 1024), (33, 8192), (300, 1024), (2048, 8192)])
+                                   (200, 1024), (33, 8192), (300, 1024), (2048, 8192), (1000, 4160),
+                                   (8192, 8192)])
 def test_dynamic_quantize_matches_oracle(orc, shape):
     # one call: S_global, quantization with it, alpha = S_global * other; small tensors
-    # take the single-launch cluster kernel, (33, 8192), (300, 1024) and (2048, 8192) the
-    # two-launch path (S_global + alpha, then the quantizer over the tiles in reverse order)
+    # take the single-launch cluster kernel, (33, 8192) and larger the two-launch path
+    # (S_global + alpha, then the quantizer over the tiles in reverse order)
     x = synth.normal_bf16(*shape, seed=28, outlier_factor=100.0)
     rows, cols = shape
     xd = to_dev_bf16(x)
@@ -258,6 +259,69 @@ def test_dynamic_quantize_matches_oracle(orc, shape):
     p_orc, s_orc = orc.quantize(fp4.NVFP4, fp4.ROWWISE, x, gs=g)
     assert np.array_equal(packed.view.cpu().numpy().reshape(rows, cols // 2), p_orc)
     assert np.array_equal(scales.view.cpu().numpy(), s_orc)
+
+
+def _dynamic_check(orc, x, ld=None):
+    rows, cols = x.shape
+    if ld is None:
+        xd = to_dev_bf16(x)
+    else:   # a strided view: the rows of a wider matrix
+        wide = np.zeros((rows, ld), dtype=np.uint16)
+        wide[:, :cols] = x
+        xd = to_dev_bf16(wide)[:, :cols]
+    p = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    s = torch.empty((fp4.fp4_scale_bytes(fp4.NVFP4, rows, cols),), dtype=torch.uint8, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    fp4.fp4_quantize_dynamic(xd, p, s, gs)
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    g = orc.global_scale(x)
+    assert np.float32(gs.item()) == np.float32(g)
+    p_orc, s_orc = orc.quantize(fp4.NVFP4, fp4.ROWWISE, x, gs=g)
+    assert np.array_equal(p.cpu().numpy(), p_orc)
+    assert np.array_equal(s.cpu().numpy(), s_orc)
+
+
+@pytest.mark.parametrize("where", ["first", "middle", "last"])
+def test_dynamic_quantize_large_amax_anywhere(orc, where):
+    # the tensor's amax in one element of the first, a middle or the last tile:
+    # every thread block's maximum must reach the reduction slot before the
+    # last one forms S_global
+    rows, cols = 1111, 2048
+    x = synth.normal_bf16(rows, cols, seed=29)
+    r, c = {"first": (0, 3), "middle": (555, 1030), "last": (rows - 1, cols - 1)}[where]
+    x[r, c] = 0x4A80   # 4194304.0, far above the rest
+    _dynamic_check(orc, x)
+
+
+def test_dynamic_quantize_large_strided_and_zero(orc):
+    x = synth.normal_bf16(700, 3072, seed=30, outlier_factor=50.0, zero_frac=0.1)
+    _dynamic_check(orc, x, ld=3200)
+    z = np.zeros((512, 4096), dtype=np.uint16)
+    _dynamic_check(orc, z)   # amax 0: S_global 1, every code and scale 0
+
+
+def test_dynamic_quantize_slot_ring_wraps(orc):
+    # more calls than the 1024 reduction slots, two tensors alternating: each
+    # call's S_global must be its own tensor's (a slot left dirty by the
+    # previous use would carry the other tensor's amax or arrivals)
+    rows, cols = 160, 8192   # above the single-cluster capacity: the S_global kernel's slots
+    xa = synth.normal_bf16(rows, cols, seed=31, outlier_factor=100.0)
+    xb = synth.normal_bf16(rows, cols, seed=32, sigma=0.01)
+    xs = [to_dev_bf16(xa), to_dev_bf16(xb)]
+    n = 1100
+    p = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    s = torch.empty((fp4.fp4_scale_bytes(fp4.NVFP4, rows, cols),), dtype=torch.uint8, device="cuda")
+    gs = torch.empty(n, dtype=torch.float32, device="cuda")
+    for i in range(n):
+        fp4.fp4_quantize_dynamic(xs[i % 2], p, s, gs[i:i + 1])
+    torch.cuda.synchronize()
+    assert fp4.fp4_get_device_status() == 0
+    ga, gb = np.float32(orc.global_scale(xa)), np.float32(orc.global_scale(xb))
+    got = gs.cpu().numpy()
+    assert np.array_equal(got[0::2], np.full(n // 2, ga)) and np.array_equal(got[1::2], np.full(n // 2, gb))
+    p_orc, s_orc = orc.quantize(fp4.NVFP4, fp4.ROWWISE, xb, gs=float(gb))
+    assert np.array_equal(p.cpu().numpy(), p_orc) and np.array_equal(s.cpu().numpy(), s_orc)
 
 
 def test_dynamic_quantize_all_zero_and_rejects_mx():
