@@ -1062,11 +1062,15 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 //                 complete on the leader's (rank 0) full[s]; the leader posts
 //                 the expected bytes of both) and the scale chunks (on the
 //                 CTA's own sf_full[s]).
-//   warp 1        MMA issue (leader CTA only): lane 0 issues the pair MMAs
-//                 and releases each stage in both CTAs (and publishes the
+//   warp 1        MMA issue (leader CTA only): passes the stage's named
+//                 barrier, then lane 0 issues the pair MMAs and releases the
+//                 stage in both CTAs (and, after a tile, publishes the
 //                 accumulator to both) with one commit that arrives on the
-//                 barrier at the same offset in each CTA.  One barrier probe
-//                 per stage, made while the stage's MMAs run.
+//                 barrier at the same offset in each CTA.  It waits on no
+//                 mbarrier inside the loop.
+//   warp 14       gatekeeper (leader CTA only): waits on the accumulator's
+//                 release and on each stage's full barrier, then lets the
+//                 MMA warp through the stage's named barrier (1 + stage).
 //   warps 2-5, 10-13  epilogue: two warps per TMEM lane quadrant, each
 //                 draining 128 of the 256 accumulator columns (tcgen05.ld,
 //                 alpha, BF16), releasing the accumulator on the leader's
@@ -1076,15 +1080,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 //                 leader's full[s], so that full[s] completes when the
 //                 operands of both CTAs have landed and both CTAs' scales are
 //                 in TMEM.
-// In the producer and MMA warps the other 31 lanes wait at __syncwarp (not at
-// a warp-aligned barrier) while lane 0 runs the loop.
+// In the producer warp the other 31 lanes wait at __syncwarp (not at a
+// warp-aligned barrier) while lane 0 runs the loop; the MMA warp runs the
+// loop with all lanes (the named barrier takes whole warps), lane 0 issuing.
 // All waits are bounded; a CTA that gives up records the error, and both
 // CTAs meet at a final cluster barrier before the pair frees its TMEM.
 // ------------------------------------------------------------------------
 constexpr int PAIR_BN = 256;                 // N of the pair tile
 constexpr int64_t kRasterGroupBytes = int64_t(32) << 20;   // A bytes per raster group
 constexpr int PAIR_BHALF = PAIR_BN / 2;      // B rows staged by each CTA
-constexpr int kPairThreads = 448;            // 14 warps, roles above
+constexpr int kPairThreads = 480;            // 15 warps, roles above
+constexpr int kGateWarp = 14;                // the gatekeeper warp of the pair kernel
 constexpr int kEpiWarps = 8;
 
 // Per stage, NVFP4 carries 4 scale chunks per 128 rows (one per K=64 MMA),
@@ -1117,6 +1123,7 @@ struct PairCfg {
     static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "tensor memory overflow");
     static_assert(NBARS * 8 + 8 <= 512, "barrier area");
     static_assert(SMEM <= 232448, "shared memory per CTA");
+    static_assert(STAGES + 1 <= 16, "one named barrier per stage (ids 1..STAGES)");
 };
 
 // 2-D TMA store of a shared-memory box to global memory (bulk-group
@@ -1145,6 +1152,17 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank)
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
+}
+
+// Hardware named barrier `id` of `count` threads: wait (all lanes of the
+// calling warp) / arrive without waiting.
+__device__ __forceinline__ void named_bar_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(int id, int count)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 __device__ __forceinline__ void cluster_sync()
@@ -1426,26 +1444,23 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issue (leader CTA only, lane 0) ----------------
-        // The tensor pipe takes a new MMA only shortly before the previous
-        // one ends, so any work of the issuing thread between two MMAs beyond
-        // about one MMA's duration leaves the pipe idle.  The per-stage work
-        // is therefore spread over the gaps between a stage's MMAs, where the
-        // thread would wait for the pipe anyway: after MMA 0 the release of
-        // the previous stage (its commit then also covers MMA 0, releasing
-        // the slot one MMA later), after MMA 1 a non-blocking probe of the
-        // next stage's barrier; between stages only the probe's result is
-        // tested (a blocking wait only if the data is late).
-        if (leader && lane == 0) {
+        // ---------------- MMA issue (leader CTA; lane 0 issues) ----------------
+        // The issuing thread touches no mbarrier inside the loop: a probe or a
+        // wait on a stage's barrier between two stages' MMAs leaves the
+        // tensor pipe idle for 40-50 of the 512 cycles a 256-deep stage takes
+        // (measured with the same loop on static operands).  The gatekeeper
+        // warp does every wait and lets this warp through stage s by the
+        // hardware named barrier 1 + s; tcgen05.fence::after_thread_sync then
+        // orders the stage's MMAs after the operand tiles and scales the
+        // gatekeeper's waits observed.  Each stage's slot is released by a
+        // commit after its MMAs, the accumulator by a commit after the tile.
+        if (leader) {
             const uint64_t adesc0 = desc_sw128(smem0);
             const uint64_t bdesc0 = desc_sw128(smem0 + C::OFF_B);
             constexpr uint32_t kDescPerStage = C::STAGE_BYTES >> 4;
             const uint32_t tsf0 = tmem_base + C::SF_COL0;
             int stage = 0;
-            uint32_t phase = 0, acc_phase = 0;
-            bool ok = true;
-            int pending = -1;   // stage whose release commit is still to be issued
-            for (int t = pair; ok && t < tiles; t += npairs) {
+            for (int t = pair; t < tiles; t += npairs) {
                 int g, tm, tn, nh;
                 locate(t, g, tm, tn, nh);
                 const Params& p = args.p[g];
@@ -1453,61 +1468,70 @@ fp4_gemm_pair_kernel(const __grid_constant__ PairArgs<NG> args)
                 const uint32_t n_mma = nh ? PAIR_BN / 2 : PAIR_BN;
                 const uint32_t idesc0 = make_idesc_pair<FMT>(0, n_mma);
                 const uint32_t idesc2 = make_idesc_pair<FMT>(2, n_mma);
-                if (!wait_fast(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY) ||
-                    !wait_fast(B_FULL(stage), phase, abort_flag, ERR_FULL)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
                 for (int ks = 0; ks < kst; ++ks) {
-                    const int nk = min(4, (p.K - ks * BK) / MMA_K);
-                    const uint64_t ad = adesc0 + (uint64_t)(stage * kDescPerStage);
-                    const uint64_t bd = bdesc0 + (uint64_t)(stage * kDescPerStage);
-                    const uint32_t tsf = tsf0 + stage * C::SF_COLS;
-                    auto mma = [&](int j) {
-                        const int chunk = MX ? (j >> 1) : j;
-                        tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j, (MX && (j & 1)) ? idesc2 : idesc0,
-                                        tsf + 4 * chunk, tsf + C::SFA_COLS + chunk * 8,
-                                        (j > 0 || ks > 0) ? 1u : 0u);
-                    };
-                    mma(0);
-                    if (pending >= 0) tc_commit_pair_both(B_EMPTY(pending));
-                    if (nk > 1) mma(1);
-                    int nstage = stage + 1;
-                    uint32_t nphase = phase;
-                    if (nstage == STAGES) {
-                        nstage = 0;
-                        nphase ^= 1u;
-                    }
-                    const bool more = ks + 1 < kst;
-                    const bool ready = more && mbar_test_wait(B_FULL(nstage), nphase);
-                    if (nk > 2) mma(2);
-                    if (nk > 3) mma(3);
-                    pending = stage;
-                    stage = nstage;
-                    phase = nphase;
-                    if (more) {
-                        if (!ready && !wait_bounded(B_FULL(stage), phase, abort_flag, ERR_FULL)) {
-                            ok = false;
-                            break;
-                        }
+                    named_bar_sync(1 + stage, 64);
+                    if (lane == 0) {
                         tc_fence_after();
+                        const int nk = min(4, (p.K - ks * BK) / MMA_K);
+                        const uint64_t ad = adesc0 + (uint64_t)(stage * kDescPerStage);
+                        const uint64_t bd = bdesc0 + (uint64_t)(stage * kDescPerStage);
+                        const uint32_t tsf = tsf0 + stage * C::SF_COLS;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (j < nk) {
+                                const int chunk = MX ? (j >> 1) : j;
+                                tc_mma_pair<MX>(tmem_base, ad + 2 * j, bd + 2 * j,
+                                                (MX && (j & 1)) ? idesc2 : idesc0, tsf + 4 * chunk,
+                                                tsf + C::SFA_COLS + chunk * 8, (j > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        tc_commit_pair_both(B_EMPTY(stage));
                     }
+                    __syncwarp();
+                    if (++stage == STAGES) stage = 0;
                 }
-                if (!ok) break;
-                tc_commit_pair_both(B_EMPTY(pending));
-                pending = -1;
-                tc_commit_pair_both(acc_full);
-                acc_phase ^= 1u;
+                if (lane == 0) tc_commit_pair_both(acc_full);
+                __syncwarp();
             }
-            if (pending >= 0) tc_commit_pair_both(B_EMPTY(pending));
-            // every pair MMA issued here has completed before the TMEM is freed
-            asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                             drain)
-                         : "memory");
-            wait_drain(drain, 0);
+            if (lane == 0) {
+                // every pair MMA issued here has completed before the TMEM is freed
+                asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                                 drain)
+                             : "memory");
+                wait_drain(drain, 0);
+            }
         }
         __syncwarp();
+    } else if (warp == kGateWarp) {
+        // ---------------- gatekeeper (leader CTA, whole warp) ----------------
+        // For each tile: the accumulator's release by both epilogues, then
+        // per stage the full barrier (both CTAs' operand tiles and the 8
+        // staging warps' scales); after each, the MMA warp is let through
+        // the stage's named barrier.  A stage is refilled only after its MMAs
+        // released it, so no named barrier has more than one arrival
+        // pending.  After a failed (timed-out) wait the warp keeps arriving
+        // without waiting, so that the MMA warp is never left blocked; the
+        // timeout is recorded in the error word.
+        if (leader) {
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int t = pair; t < tiles; t += npairs) {
+                int g, tm, tn, nh;
+                locate(t, g, tm, tn, nh);
+                const int kst = args.p[g].ks_total;
+                if (ok && !warp_wait(acc_empty, acc_phase ^ 1u, abort_flag, ERR_ACC_EMPTY)) ok = false;
+                for (int ks = 0; ks < kst; ++ks) {
+                    if (ok && !warp_wait(B_FULL(stage), phase, abort_flag, ERR_FULL)) ok = false;
+                    named_bar_arrive(1 + stage, 64);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                acc_phase ^= 1u;
+            }
+        }
     } else if (warp < 6 || warp >= 10) {
         // ---------------- epilogue (warps 2..5 and 10..13, both CTAs) ----------------
         const int q = warp & 3;                      // TMEM lane quadrant
