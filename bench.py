@@ -178,6 +178,50 @@ def _qbufs(fmt, rows, K, dev):
             torch.empty((fp4.fp4_scale_bytes(fmt, rows, K),), dtype=torch.uint8, device=dev))
 
 
+class E2EPipeline:
+    """Steps through the public API with each step's host-to-device copy,
+    its compute and its device-to-host copy on three streams, two slots of
+    device buffers: step i's input copy and step i-1's result copy run while
+    step i's (or i-1's) kernels do, on both directions of the PCIe link.
+    Events order, for each slot, the input copy after the compute that last
+    read the slot, the compute after its input and after the result copy
+    that last read the slot's D, and the result copy after the compute."""
+
+    def __init__(self, wl, dev):
+        self.wl = wl
+        self.streams = [torch.cuda.Stream(dev) for _ in range(3)]   # h2d, compute, d2h
+        self.ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "comp", "d2h")}
+        self.used = [False, False]
+
+    def step(self, i):
+        j = i % 2
+        sh, sc, sd = self.streams
+        with torch.cuda.stream(sh):
+            if self.used[j]:
+                sh.wait_event(self.ev["comp"][j])
+            self.wl.e2e_h2d(j)
+            self.ev["h2d"][j].record(sh)
+        with torch.cuda.stream(sc):
+            sc.wait_event(self.ev["h2d"][j])
+            if self.used[j]:
+                sc.wait_event(self.ev["d2h"][j])
+            self.wl.e2e_compute(j)
+            self.ev["comp"][j].record(sc)
+        with torch.cuda.stream(sd):
+            sd.wait_event(self.ev["comp"][j])
+            self.wl.e2e_d2h(j)
+            self.ev["d2h"][j].record(sd)
+        self.used[j] = True
+
+    def begin(self, ev):
+        for s in self.streams:
+            s.wait_event(ev)
+
+    def end(self, stream):
+        for s in self.streams:
+            stream.wait_stream(s)
+
+
 class SquareWorkload(Workload):
     """Quantize A and B (rowwise, along K) and D = A_hat B_hat^T, M=N=K=n."""
 
@@ -223,29 +267,43 @@ class SquareWorkload(Workload):
     def value(self, sec_per_step):
         return self.flops / sec_per_step / 1e12
 
+    # ---- end to end through the public API (three phases per step, on two
+    # slots of device buffers; E2EPipeline overlaps them across steps) ------
     def e2e_setup(self, dev):
         A, B = self.host
+        fmt, n = self.fmt, self.n
         self.hA = synth.bits_to_torch(A).pin_memory()
         self.hB = synth.bits_to_torch(B).pin_memory()
-        self.hD = torch.empty((self.n, self.n), dtype=torch.bfloat16).pin_memory()
+        self.hD = torch.empty((n, n), dtype=torch.bfloat16).pin_memory()
+        self.e2e_slots = []
+        for _ in range(2):
+            sl = {"A": torch.empty((n, n), dtype=torch.bfloat16, device=dev),
+                  "B": torch.empty((n, n), dtype=torch.bfloat16, device=dev),
+                  "D": torch.empty((n, n), dtype=torch.bfloat16, device=dev)}
+            sl["pA"], sl["sA"] = _qbufs(fmt, n, n, dev)
+            sl["pB"], sl["sB"] = _qbufs(fmt, n, n, dev)
+            sl["g"] = torch.empty(3, dtype=torch.float32, device=dev)   # gA, gB, alpha
+            self.e2e_slots.append(sl)
         return 2 * self.hA.numel() * 2, self.hD.numel() * 2
 
-    def e2e_step(self, dev):
-        fmt, n = self.fmt, self.n
-        Ad = self.hA.to(dev, non_blocking=True)
-        Bd = self.hB.to(dev, non_blocking=True)
+    def e2e_h2d(self, j):
+        sl = self.e2e_slots[j]
+        sl["A"].copy_(self.hA, non_blocking=True)
+        sl["B"].copy_(self.hB, non_blocking=True)
+
+    def e2e_compute(self, j):
+        fmt, n, sl = self.fmt, self.n, self.e2e_slots[j]
         if fmt == fp4.NVFP4:
-            gA = torch.empty(1, dtype=torch.float32, device=dev)
-            gB = torch.empty(1, dtype=torch.float32, device=dev)
-            al = torch.empty(1, dtype=torch.float32, device=dev)
-            fp4.fp4_compute_global_scales_pair(Ad, Bd, gA, gB, al)
+            gA, gB, al = sl["g"][0:1], sl["g"][1:2], sl["g"][2:3]
+            fp4.fp4_compute_global_scales_pair(sl["A"], sl["B"], gA, gB, al)
         else:
             gA = gB = al = None
-        pA, sA = _qbufs(fmt, n, n, dev)
-        pB, sB = _qbufs(fmt, n, n, dev)
-        fp4.fp4_quantize_batch(fmt, [(Ad, pA, sA, gA), (Bd, pB, sB, gB)])
-        D = fp4.gemm(fmt, pA, sA, pB, sB, n, alpha=al, kernel=fp4.GEMM_PREFILL)
-        self.hD.copy_(D, non_blocking=True)
+        fp4.fp4_quantize_batch(fmt, [(sl["A"], sl["pA"], sl["sA"], gA), (sl["B"], sl["pB"], sl["sB"], gB)])
+        fp4.gemm(fmt, sl["pA"], sl["sA"], sl["pB"], sl["sB"], n, alpha=al, kernel=fp4.GEMM_PREFILL,
+                 out=sl["D"])
+
+    def e2e_d2h(self, j):
+        self.hD.copy_(self.e2e_slots[j]["D"], non_blocking=True)
 
     def oracle_sample(self, orc, r):
         """Oracle on an r x r sub-problem of the step: S_global passes (NVFP4)
@@ -523,25 +581,41 @@ class PrefillWorkload(Workload):
     def value(self, sec_per_step):
         return self.flops / sec_per_step / 1e12
 
-    # ---- end to end through the public API --------------------------------
+    # ---- end to end through the public API (three phases per step, on two
+    # slots of device buffers; E2EPipeline overlaps them across steps) ------
+    # The step's activation arrives from pinned host memory; the resident
+    # quantized weights are the layer's parameters; D goes back to the host.
     def e2e_setup(self, dev):
         A, _ = self.host
+        M, N, K = self.M, self.N, self.K
         self.hA = synth.bits_to_torch(A).pin_memory()
-        self.hD = torch.empty((self.M, self.N), dtype=torch.bfloat16).pin_memory()
+        self.hD = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        self.e2e_slots = []
+        for _ in range(2):
+            sl = {"A": torch.empty((M, K), dtype=torch.bfloat16, device=dev),
+                  "D": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                  "g": torch.empty(2, dtype=torch.float32, device=dev)}   # gA, alpha
+            sl["pA"], sl["sA"] = _qbufs(fp4.NVFP4, M, K, dev)
+            self.e2e_slots.append(sl)
         return self.hA.numel() * 2, self.hD.numel() * 2
 
-    def e2e_step(self, dev):
-        # the step's activation arrives from pinned host memory; the resident
-        # quantized weights are the layer's parameters; D goes back to the host
-        M, N, K = self.M, self.N, self.K
+    def e2e_h2d(self, j):
+        self.e2e_slots[j]["A"].copy_(self.hA, non_blocking=True)
+
+    def e2e_compute(self, j):
+        K, sl = self.K, self.e2e_slots[j]
         pW, sW, gW = self.weights
-        Ad = self.hA.to(dev, non_blocking=True)
-        gA = torch.empty(1, dtype=torch.float32, device=dev)
-        al = torch.empty(1, dtype=torch.float32, device=dev)
-        pA, sA = _qbufs(fp4.NVFP4, M, K, dev)
-        fp4.fp4_quantize_dynamic(Ad, pA, sA, gA, gW, al)
-        D = fp4.gemm(fp4.NVFP4, pA, sA, pW, sW, K, alpha=al, kernel=fp4.GEMM_PREFILL)
-        self.hD.copy_(D, non_blocking=True)
+        fp4.fp4_quantize_dynamic(sl["A"], sl["pA"], sl["sA"], sl["g"][0:1], gW, sl["g"][1:2])
+        fp4.gemm(fp4.NVFP4, sl["pA"], sl["sA"], pW, sW, K, alpha=sl["g"][1:2], kernel=fp4.GEMM_PREFILL,
+                 out=sl["D"])
+
+    def e2e_d2h(self, j):
+        self.hD.copy_(self.e2e_slots[j]["D"], non_blocking=True)
+
+    def e2e_expected(self):
+        """The device path's D for the same activation (the timed graph's
+        output), which the host copy of the last end-to-end step must equal."""
+        return self.bufs[0][7]
 
     # ---- the oracle on a bounded sample of the step ------------------------
     def oracle_sample(self, orc, tiles, seed=0):
@@ -909,20 +983,30 @@ def main():
     e2e = None
     if not args.no_e2e and hasattr(wl, "e2e_setup"):
         hb, db = wl.e2e_setup(dev)
-        for _ in range(3):
-            wl.e2e_step(dev)
+        pipe = E2EPipeline(wl, dev)
+        for i in range(3):
+            pipe.step(i)
         torch.cuda.synchronize()
         n_e2e = 20
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(n_e2e):
-            wl.e2e_step(dev)
+        pipe.begin(a)
+        for i in range(n_e2e):
+            pipe.step(i)
+        pipe.end(stream)
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, dist, dev)
         e2e = {"value": job_throughput(wl.value(e_ms / 1e3), world, 1.0), "unit": wl.unit,
                "h2d_bytes_per_step": hb,
-               "d2h_bytes_per_step": db, "ms_per_step": e_ms}
+               "d2h_bytes_per_step": db, "ms_per_step": e_ms,
+               "pipeline": "3 streams, 2 buffer slots: step i's input copy and step i-1's result copy "
+                           "overlap the kernels"}
+        if hasattr(wl, "e2e_expected"):
+            same = bool(torch.equal(wl.hD, wl.e2e_expected().cpu()))
+            e2e["result_matches_device_path"] = same
+            if not same:
+                raise SystemExit("end-to-end result differs from the device path's")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and hasattr(wl, "cpu_baseline"):
