@@ -187,27 +187,32 @@ class E2EPipeline:
     read the slot, the compute after its input and after the result copy
     that last read the slot's D, and the result copy after the compute."""
 
-    def __init__(self, wl, dev):
+    def __init__(self, wl, dev, new_stream=None, new_event=None, on_stream=None):
+        # the CUDA stream/event constructors and stream context (replaceable
+        # by recording fakes that check the ordering without a device)
+        new_stream = new_stream or (lambda: torch.cuda.Stream(dev))
+        new_event = new_event or torch.cuda.Event
+        self.on_stream = on_stream or torch.cuda.stream
         self.wl = wl
-        self.streams = [torch.cuda.Stream(dev) for _ in range(3)]   # h2d, compute, d2h
-        self.ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("h2d", "comp", "d2h")}
+        self.streams = [new_stream() for _ in range(3)]   # h2d, compute, d2h
+        self.ev = {k: [new_event() for _ in range(2)] for k in ("h2d", "comp", "d2h")}
         self.used = [False, False]
 
     def step(self, i):
         j = i % 2
         sh, sc, sd = self.streams
-        with torch.cuda.stream(sh):
+        with self.on_stream(sh):
             if self.used[j]:
                 sh.wait_event(self.ev["comp"][j])
             self.wl.e2e_h2d(j)
             self.ev["h2d"][j].record(sh)
-        with torch.cuda.stream(sc):
+        with self.on_stream(sc):
             sc.wait_event(self.ev["h2d"][j])
             if self.used[j]:
                 sc.wait_event(self.ev["d2h"][j])
             self.wl.e2e_compute(j)
             self.ev["comp"][j].record(sc)
-        with torch.cuda.stream(sd):
+        with self.on_stream(sd):
             sd.wait_event(self.ev["comp"][j])
             self.wl.e2e_d2h(j)
             self.ev["d2h"][j].record(sd)
